@@ -1,0 +1,206 @@
+/*
+ * dsa.h -- C ABI of the DeepSeek Sparse Attention (DSA) forward path on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * DSA replaces dense causal attention by three steps per query token
+ * (DeepSeek-V3.2-Exp report read-through on 53ai.com, section "Innovative
+ * architecture: core design of DSA", and its Figure 1):
+ *   1. a lightning indexer scores the query against every preceding token:
+ *        I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s]),   s <= t,
+ *      multi-head and ReLU-gated, with FP8 inputs;
+ *   2. fine-grained selection keeps the k best-scoring tokens (k = 2048 in
+ *      DeepSeek-V3.2: paperbridge.wiki summary, section "DeepSeek Sparse
+ *      Attention"; juhe.plus read-through, step 2);
+ *   3. attention runs in MLA's MQA mode -- one latent KV row shared by all
+ *      query heads -- over the selected rows only.
+ *
+ * Conventions shared by every call
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller. The
+ *     library never allocates device memory on these paths; scratch space is
+ *     the caller's workspace, sized by dsa_workspace_size().
+ *   - Every call is asynchronous on the given CUDA stream (a cudaStream_t;
+ *     NULL is the legacy default stream). Host-side argument checks run before
+ *     any launch and return an error without launching anything.
+ *   - Errors found on the device (an index or page id out of range, a bounded
+ *     wait that ran out) are recorded in a per-device status word; read it
+ *     with dsa_check_status(), which synchronises the stream. Device code
+ *     never traps: bad indices are skipped (treated as masked) and reported.
+ *   - Positions. CONTIGUOUS layout: keys are rows 0..n_keys-1 of one
+ *     sequence and query i sits at position n_keys - n_q + i (n_q == n_keys is
+ *     a plain prefill). PAGED layout: query b belongs to sequence b, whose
+ *     ctx_lens[b] cached tokens include the query token, so the query sits at
+ *     position ctx_lens[b] - 1. In both cases the query sees keys 0..pos
+ *     (inclusive: the pages say "preceding tokens"; the token itself is kept so
+ *     that every row has at least one key).
+ *   - Supported combinations (others return DSA_ERR_UNSUPPORTED):
+ *       E4M3 indexer (H_I=64, d_I=128) + BF16 attention (H=128, d_qk=576,
+ *       d_v=512, V = first 512 columns of the KV row), CONTIGUOUS or PAGED
+ *       with 64-token pages;
+ *       F32 indexer (H_I<=64, d_I<=128, d_I%4==0) + F32 attention (H<=128,
+ *       d_qk<=256, d_v<=256, separate V allowed), CONTIGUOUS only.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+/* A cudaStream_t. */
+typedef struct CUstream_st* dsa_stream_t;
+
+typedef enum dsa_status {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,          /* null pointer, bad size/stride/alignment, k out of [1,2048] */
+  DSA_ERR_UNSUPPORTED = 2,          /* dtype/dims/layout combination not built */
+  DSA_ERR_WORKSPACE_TOO_SMALL = 3,  /* ws_bytes < dsa_workspace_size() */
+  DSA_ERR_CUDA = 4,                 /* a CUDA runtime call failed; see dsa_last_cuda_error() */
+  DSA_ERR_DEVICE_BOUNDS = 5,        /* device saw an index/page id out of range (skipped) */
+  DSA_ERR_TIMEOUT = 6               /* a bounded device wait ran out; results are invalid */
+} dsa_status;
+
+typedef enum dsa_dtype {
+  DSA_F32 = 0,   /* float32 */
+  DSA_E4M3 = 1,  /* OCP FP8 e4m3 codes (uint8) + one float32 scale per token */
+  DSA_BF16 = 2   /* bfloat16 */
+} dsa_dtype;
+
+typedef enum dsa_kv_kind {
+  DSA_KV_CONTIGUOUS = 0,
+  DSA_KV_PAGED = 1
+} dsa_kv_kind;
+
+/* Where the keys live. For PAGED, logical token p of sequence b is slot
+ * p % page_size of page block_table[b * ld_block_table + p / page_size]. */
+typedef struct dsa_kv_layout {
+  int32_t kind;                 /* dsa_kv_kind */
+  int32_t page_size;            /* PAGED: tokens per page, must be 64 */
+  const int32_t* block_table;   /* PAGED: device [n_q, ld_block_table] page ids */
+  int64_t ld_block_table;       /* PAGED: elements between rows of block_table */
+  int32_t max_pages;            /* PAGED: columns of block_table usable per row */
+  int32_t num_pages;            /* PAGED: pages in the caches (page ids must be < this) */
+  const int32_t* ctx_lens;      /* PAGED: device [n_q] cached tokens per sequence, in [1, max_pages*page_size] */
+} dsa_kv_layout;
+
+/* Indexer inputs (step 1). Token-major rows; all strides in ELEMENTS.
+ * E4M3: q/k hold e4m3 codes, the real value of an entry is
+ *       decode(code) * q_scale[token] (resp. k_scale[key token]), scales > 0.
+ * F32 : q/k hold the real values; q_scale/k_scale must be NULL. */
+typedef struct dsa_indexer_in {
+  int32_t dtype;        /* DSA_E4M3 or DSA_F32 */
+  int32_t n_q;          /* query tokens */
+  int32_t n_keys;       /* CONTIGUOUS: key tokens (>= n_q); PAGED: ignored */
+  int32_t heads;        /* H_I */
+  int32_t dim;          /* d_I */
+  const void* q;        /* [n_q, heads, dim]; heads contiguous within a token */
+  int64_t ld_q;         /* elements between query tokens (>= heads*dim) */
+  const float* q_scale; /* E4M3: [n_q] */
+  const void* k;        /* CONTIGUOUS: [n_keys, dim]; PAGED: [num_pages, page_size, dim] */
+  int64_t ld_k;         /* elements between key tokens (>= dim) */
+  const float* k_scale; /* E4M3: CONTIGUOUS [n_keys]; PAGED [num_pages * page_size] */
+  const float* w;       /* [n_q, heads] per-query head weights */
+  int64_t ld_w;         /* elements between query tokens of w (>= heads) */
+  dsa_kv_layout kv;
+} dsa_indexer_in;
+
+/* Attention inputs (step 3). V defaults to the first d_v columns of each KV
+ * row (MLA latent); a separate V is accepted for F32 only. */
+typedef struct dsa_attn_in {
+  int32_t dtype;        /* DSA_BF16 or DSA_F32 */
+  int32_t n_q;          /* query tokens (same as the indexer's) */
+  int32_t n_keys;       /* CONTIGUOUS: KV rows; PAGED: ignored */
+  int32_t heads;        /* H */
+  int32_t d_qk;         /* key/query width */
+  int32_t d_v;          /* value width */
+  float scale;          /* softmax scale on q.k (e.g. 1/sqrt(d_qk)) */
+  const void* q;        /* [n_q, heads, d_qk], heads contiguous */
+  int64_t ld_q;         /* elements between query tokens (>= heads*d_qk) */
+  const void* kv;       /* CONTIGUOUS: [n_keys, d_qk]; PAGED: [num_pages, page_size, d_qk] */
+  int64_t ld_kv;        /* elements between KV rows (>= d_qk) */
+  const void* v;        /* NULL, or F32 only: [n_keys, d_v] */
+  int64_t ld_v;
+  dsa_kv_layout kv_layout;
+} dsa_attn_in;
+
+typedef enum dsa_op {
+  DSA_OP_INDEXER_SCORES = 0,
+  DSA_OP_TOPK = 1,
+  DSA_OP_SPARSE_MQA = 2,
+  DSA_OP_FORWARD = 3
+} dsa_op;
+
+/* Step 1 alone: lightning-indexer scores for selected query rows.
+ * Row r of `scores` (row stride ld_scores floats) belongs to query
+ * rows ? rows[r] : r (device array, values in [0, n_q)). Columns 0..n_cols-1
+ * are written: the score for keys s <= pos(query), -INFINITY for s > pos.
+ * Scores are float32 and bit-identical to those the fused dsa_forward ranks.
+ * Requires n_cols >= 1, ld_scores >= n_cols; for PAGED n_cols <=
+ * max_pages*page_size. Workspace: dsa_workspace_size(DSA_OP_INDEXER_SCORES). */
+DSA_API dsa_status dsa_indexer_scores(const dsa_indexer_in* in, const int32_t* rows,
+                                      int32_t n_rows, float* scores, int64_t ld_scores,
+                                      int32_t n_cols, void* ws, size_t ws_bytes,
+                                      dsa_stream_t stream);
+
+/* Step 2 alone: exact top-k of each score row.
+ * Row r considers scores[r*ld_scores + s] for s in [0, row_pos[r]] (device
+ * array). It keeps the min(k, row_pos[r]+1) entries with the largest score,
+ * ties to the lower s, -0.0 equal to +0.0, NaN below every number, and writes
+ * their s in ascending order to idx[r*ld_idx + 0..], padding with -1 up to k.
+ * Needs no workspace. 1 <= k <= 2048; 0 <= row_pos[r] < 2^31-1. */
+DSA_API dsa_status dsa_topk(const float* scores, int64_t ld_scores, const int32_t* row_pos,
+                            int32_t n_rows, int32_t k, int32_t* idx, int64_t ld_idx,
+                            dsa_stream_t stream);
+
+/* Step 3 alone: sparse MQA attention.
+ * For query i, idx[i*ld_idx + 0..k-1] lists key positions (logical positions
+ * for PAGED); entries < 0 are skipped, entries > pos(query) are reported as
+ * DSA_ERR_DEVICE_BOUNDS and skipped. Every row must hold at least one valid
+ * entry. out: [n_q, heads, d_v] contiguous, same dtype as q; lse: [n_q, heads]
+ * float32 natural-log log-sum-exp of the scaled logits (may be NULL).
+ * Workspace: dsa_workspace_size(DSA_OP_SPARSE_MQA). */
+DSA_API dsa_status dsa_sparse_mqa_fwd(const dsa_attn_in* in, const int32_t* idx, int64_t ld_idx,
+                                      int32_t k, void* out, float* lse, void* ws,
+                                      size_t ws_bytes, dsa_stream_t stream);
+
+/* Steps 1-3 fused: indexer -> top-k -> sparse attention without ever holding
+ * the n_q x n_keys score matrix (prefill streams the indexer over bounded
+ * blocks of queries). idx_out (nullable, [n_q, k] int32) receives the
+ * selection, identical to dsa_topk(dsa_indexer_scores(...)).
+ * Workspace: dsa_workspace_size(DSA_OP_FORWARD). */
+DSA_API dsa_status dsa_forward(const dsa_indexer_in* indexer, const dsa_attn_in* attn,
+                               int32_t k, int32_t* idx_out, void* out, float* lse,
+                               void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Workspace bytes for `op` with these inputs (arguments an op does not use may
+ * be NULL/0). The workspace must be 256-byte aligned device memory. */
+DSA_API dsa_status dsa_workspace_size(int32_t op, const dsa_indexer_in* indexer,
+                                      const dsa_attn_in* attn, int32_t n_rows, int32_t n_cols,
+                                      int32_t k, size_t* bytes);
+
+/* Synchronises `stream`, returns the first device-side error recorded on the
+ * current device since the last call (DSA_OK if none) and clears it. */
+DSA_API dsa_status dsa_check_status(dsa_stream_t stream);
+
+/* Static description of a status code. */
+DSA_API const char* dsa_status_string(dsa_status status);
+
+/* The cudaError_t value behind the last DSA_ERR_CUDA on this thread (0 if none). */
+DSA_API int32_t dsa_last_cuda_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+DSA_API int32_t dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

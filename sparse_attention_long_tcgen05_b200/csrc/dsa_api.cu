@@ -1,0 +1,514 @@
+// dsa_api.cu -- the C ABI declared in include/dsa.h: host-side validation,
+// TMA tensor-map encoding, workspace carving and stream-ordered launches of the
+// DSA kernels. Nothing here computes a step of the method; every step runs in
+// the kernels. No device memory is allocated on these paths.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "dsa.h"
+#include "dsa_kernels.h"
+
+// Per-device status word written by the kernels' checks (first error wins).
+__device__ int g_dsa_status;
+
+namespace {
+
+thread_local int32_t t_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+constexpr int kKMax = 2048;
+constexpr int kPage = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  int* status = nullptr;
+  int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+dsa_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int32_t>(e);
+  return DSA_ERR_CUDA;
+}
+
+#define DSA_TRY_CUDA(expr)                          \
+  do {                                              \
+    cudaError_t e_ = (expr);                        \
+    if (e_ != cudaSuccess) return cuda_fail(e_);    \
+  } while (0)
+
+#define DSA_TRY(expr)                               \
+  do {                                              \
+    dsa_status s_ = (expr);                         \
+    if (s_ != DSA_OK) return s_;                    \
+  } while (0)
+
+// Device status word address and SM count of the current device (set up once
+// per device, with that device current).
+dsa_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  DSA_TRY_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    void* p = nullptr;
+    DSA_TRY_CUDA(cudaGetSymbolAddress(&p, g_dsa_status));
+    DSA_TRY_CUDA(cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev));
+    int major = 0, minor = 0;
+    DSA_TRY_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    DSA_TRY_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    if (major != 10 || minor != 0) return DSA_ERR_UNSUPPORTED;   // sm_100a only
+    d.status = static_cast<int*>(p);
+    d.init = true;
+  }
+  *out = &d;
+  return DSA_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// rank-D tiled map; dims/box innermost first; strides (bytes) of dims 1..D-1.
+dsa_status make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
+                    const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+                    CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t d[5], s[4];
+  cuuint32_t b[5], e[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    e[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) s[i] = strides[i];
+  CUresult r = fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, s, b, e,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- validation
+
+dsa_status check_layout(const dsa_kv_layout& kv, int32_t n_q, int32_t n_keys) {
+  if (kv.kind == DSA_KV_CONTIGUOUS) {
+    if (n_q < 1 || n_keys < n_q) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+  }
+  if (kv.kind != DSA_KV_PAGED) return DSA_ERR_INVALID_ARG;
+  if (kv.page_size != kPage) return DSA_ERR_UNSUPPORTED;
+  if (n_q < 1 || kv.block_table == nullptr || kv.ctx_lens == nullptr || kv.max_pages < 1 ||
+      kv.num_pages < 1 || kv.ld_block_table < kv.max_pages)
+    return DSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(kv.max_pages) * kPage > 0x7fffffffLL) return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+dsa::KeySide key_side(const dsa_kv_layout& kv, int32_t n_q, int32_t n_keys) {
+  dsa::KeySide k{};
+  k.paged = kv.kind == DSA_KV_PAGED;
+  k.n_q = n_q;
+  k.n_keys = n_keys;
+  k.block_table = kv.block_table;
+  k.ld_block_table = kv.ld_block_table;
+  k.max_pages = kv.max_pages;
+  k.num_pages = kv.num_pages;
+  k.ctx_lens = kv.ctx_lens;
+  return k;
+}
+
+bool is_fp8_indexer(const dsa_indexer_in& in) {
+  return in.dtype == DSA_E4M3 && in.heads == 64 && in.dim == 128;
+}
+
+dsa_status check_indexer(const dsa_indexer_in* in) {
+  if (in == nullptr) return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_layout(in->kv, in->n_q, in->n_keys));
+  if (in->q == nullptr || in->k == nullptr || in->w == nullptr) return DSA_ERR_INVALID_ARG;
+  if (in->heads < 1 || in->dim < 1) return DSA_ERR_INVALID_ARG;
+  if (in->ld_q < static_cast<int64_t>(in->heads) * in->dim || in->ld_k < in->dim ||
+      in->ld_w < in->heads)
+    return DSA_ERR_INVALID_ARG;
+  if (in->dtype == DSA_E4M3) {
+    if (!is_fp8_indexer(*in)) return DSA_ERR_UNSUPPORTED;
+    if (in->q_scale == nullptr || in->k_scale == nullptr) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(in->q) || !aligned16(in->k) || in->ld_q % 16 || in->ld_k % 16)
+      return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+  }
+  if (in->dtype == DSA_F32) {
+    if (in->kv.kind != DSA_KV_CONTIGUOUS) return DSA_ERR_UNSUPPORTED;
+    if (in->heads > 64 || in->dim > 128 || in->dim % 4) return DSA_ERR_UNSUPPORTED;
+    if (in->q_scale != nullptr || in->k_scale != nullptr) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(in->k) || in->ld_k % 4) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+  }
+  return DSA_ERR_UNSUPPORTED;
+}
+
+bool is_bf16_attn(const dsa_attn_in& in) {
+  return in.dtype == DSA_BF16 && in.heads == 128 && in.d_qk == 576 && in.d_v == 512;
+}
+
+dsa_status check_attn(const dsa_attn_in* in) {
+  if (in == nullptr) return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_layout(in->kv_layout, in->n_q, in->n_keys));
+  if (in->q == nullptr || in->kv == nullptr) return DSA_ERR_INVALID_ARG;
+  if (in->heads < 1 || in->d_qk < 1 || in->d_v < 1) return DSA_ERR_INVALID_ARG;
+  if (!(in->scale > 0.f) || !std::isfinite(in->scale)) return DSA_ERR_INVALID_ARG;
+  if (in->ld_q < static_cast<int64_t>(in->heads) * in->d_qk || in->ld_kv < in->d_qk)
+    return DSA_ERR_INVALID_ARG;
+  if (in->dtype == DSA_BF16) {
+    if (!is_bf16_attn(*in) || in->v != nullptr) return DSA_ERR_UNSUPPORTED;
+    if (!aligned16(in->q) || !aligned16(in->kv) || (in->ld_q * 2) % 16 || (in->ld_kv * 2) % 16)
+      return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+  }
+  if (in->dtype == DSA_F32) {
+    if (in->kv_layout.kind != DSA_KV_CONTIGUOUS) return DSA_ERR_UNSUPPORTED;
+    if (in->heads > 128 || in->d_qk > 256 || in->d_v > 256) return DSA_ERR_UNSUPPORTED;
+    if (in->v == nullptr && in->d_v > in->d_qk) return DSA_ERR_INVALID_ARG;
+    if (in->v != nullptr && in->ld_v < in->d_v) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+  }
+  return DSA_ERR_UNSUPPORTED;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Query rows per indexer launch inside the fused prefill: the score block of
+// one launch (rows x keys floats) stays within 64 MiB, half of the 126 MB L2.
+int32_t forward_chunk_rows(int32_t n_q, int32_t n_cols) {
+  int64_t c = (int64_t(16) << 20) / (n_cols > 0 ? n_cols : 1);
+  c = c < 128 ? 128 : c;
+  c = (c / 4) * 4;
+  return c > n_q ? n_q : static_cast<int32_t>(c);
+}
+
+struct ForwardPlan {
+  int32_t n_cols;      // columns of a score row
+  int32_t chunk;       // query rows per indexer launch
+  size_t scores_bytes;
+  size_t idx_bytes;
+};
+
+ForwardPlan forward_plan(const dsa_indexer_in& ind, int32_t k) {
+  ForwardPlan p{};
+  if (ind.kv.kind == DSA_KV_PAGED) {
+    p.n_cols = ind.kv.max_pages * kPage;
+    p.chunk = ind.n_q;
+  } else {
+    p.n_cols = ind.n_keys;
+    p.chunk = forward_chunk_rows(ind.n_q, ind.n_keys);
+  }
+  p.scores_bytes = round256(static_cast<size_t>(p.chunk) * p.n_cols * sizeof(float));
+  p.idx_bytes = round256(static_cast<size_t>(ind.n_q) * k * sizeof(int32_t));
+  return p;
+}
+
+// ---------------------------------------------------------------- launchers
+
+dsa_status run_indexer(const dsa_indexer_in& in, const int32_t* rows, int32_t q_base,
+                       int32_t n_rows, float* scores, int64_t ld_scores, int32_t n_cols,
+                       int write_masked, DeviceInfo* dev, cudaStream_t stream) {
+  const dsa::KeySide ks = key_side(in.kv, in.n_q, in.n_keys);
+  if (in.dtype == DSA_E4M3) {
+    dsa::IndexerFp8Args a{};
+    {
+      const uint64_t dims[3] = {128, 64, static_cast<uint64_t>(in.n_q)};
+      const uint64_t strides[2] = {128, static_cast<uint64_t>(in.ld_q)};
+      const uint32_t box[3] = {128, 64, 1};
+      DSA_TRY(make_map(&a.map_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, in.q, dims, strides, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B));
+    }
+    {
+      const uint64_t rows_k = ks.paged ? static_cast<uint64_t>(in.kv.num_pages) * kPage
+                                       : static_cast<uint64_t>(in.n_keys);
+      const uint64_t dims[2] = {128, rows_k};
+      const uint64_t strides[1] = {static_cast<uint64_t>(in.ld_k)};
+      const uint32_t box[2] = {128, ks.paged ? 64u : 128u};
+      DSA_TRY(make_map(&a.map_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, in.k, dims, strides, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B));
+    }
+    a.q_scale = in.q_scale;
+    a.w = in.w;
+    a.ld_w = in.ld_w;
+    a.k_scale = in.k_scale;
+    a.keys = ks;
+    a.qr = {rows, q_base, n_rows};
+    a.scores = scores;
+    a.ld_scores = ld_scores;
+    a.n_cols = n_cols;
+    a.write_masked = write_masked;
+    a.status = dev->status;
+    DSA_TRY_CUDA(dsa::launch_indexer_fp8(a, dev->num_sms, stream));
+    return DSA_OK;
+  }
+  dsa::IndexerF32Args a{};
+  a.q = static_cast<const float*>(in.q);
+  a.ld_q = in.ld_q;
+  a.k = static_cast<const float*>(in.k);
+  a.ld_k = in.ld_k;
+  a.w = in.w;
+  a.ld_w = in.ld_w;
+  a.heads = in.heads;
+  a.dim = in.dim;
+  a.keys = ks;
+  a.qr = {rows, q_base, n_rows};
+  a.scores = scores;
+  a.ld_scores = ld_scores;
+  a.n_cols = n_cols;
+  a.status = dev->status;
+  DSA_TRY_CUDA(dsa::launch_indexer_f32(a, stream));
+  return DSA_OK;
+}
+
+dsa_status run_topk(const float* scores, int64_t ld_scores, const int32_t* row_pos,
+                    int32_t pos_minus, int32_t pos_base, int32_t n_rows, int32_t k, int32_t* idx, int64_t ld_idx,
+                    DeviceInfo* dev, cudaStream_t stream) {
+  dsa::TopkArgs a{};
+  a.scores = scores;
+  a.ld_scores = ld_scores;
+  a.row_pos = row_pos;
+  a.pos_minus = pos_minus;
+  a.pos_base = pos_base;
+  a.n_rows = n_rows;
+  a.k = k;
+  a.idx = idx;
+  a.ld_idx = ld_idx;
+  a.status = dev->status;
+  DSA_TRY_CUDA(dsa::launch_topk(a, stream));
+  return DSA_OK;
+}
+
+dsa_status run_attn(const dsa_attn_in& in, const int32_t* idx, int64_t ld_idx, int32_t k,
+                    void* out, float* lse, DeviceInfo* dev, cudaStream_t stream) {
+  const dsa::KeySide ks = key_side(in.kv_layout, in.n_q, in.n_keys);
+  if (in.dtype == DSA_BF16) {
+    dsa::AttnBf16Args a{};
+    {
+      const uint64_t dims[3] = {576, 128, static_cast<uint64_t>(in.n_q)};
+      const uint64_t strides[2] = {576 * 2, static_cast<uint64_t>(in.ld_q) * 2};
+      const uint32_t box[3] = {64, 128, 1};
+      DSA_TRY(make_map(&a.map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, in.q, dims, strides, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B));
+    }
+    {
+      const uint64_t rows_kv = ks.paged ? static_cast<uint64_t>(in.kv_layout.num_pages) * kPage
+                                        : static_cast<uint64_t>(in.n_keys);
+      const uint64_t dims[2] = {576, rows_kv};
+      const uint64_t strides[1] = {static_cast<uint64_t>(in.ld_kv) * 2};
+      const uint32_t box[2] = {64, 1};
+      DSA_TRY(make_map(&a.map_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, in.kv, dims, strides,
+                       box, CU_TENSOR_MAP_SWIZZLE_128B));
+    }
+    a.idx = idx;
+    a.ld_idx = ld_idx;
+    a.k = k;
+    a.keys = ks;
+    a.scale_log2 = in.scale * 1.4426950408889634f;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.lse = lse;
+    a.status = dev->status;
+    DSA_TRY_CUDA(dsa::launch_attn_bf16(a, stream));
+    return DSA_OK;
+  }
+  dsa::AttnF32Args a{};
+  a.q = static_cast<const float*>(in.q);
+  a.ld_q = in.ld_q;
+  a.kv = static_cast<const float*>(in.kv);
+  a.ld_kv = in.ld_kv;
+  a.v = static_cast<const float*>(in.v);
+  a.ld_v = in.ld_v;
+  a.heads = in.heads;
+  a.d_qk = in.d_qk;
+  a.d_v = in.d_v;
+  a.scale = in.scale;
+  a.idx = idx;
+  a.ld_idx = ld_idx;
+  a.k = k;
+  a.keys = ks;
+  a.out = static_cast<float*>(out);
+  a.lse = lse;
+  a.status = dev->status;
+  DSA_TRY_CUDA(dsa::launch_attn_f32(a, stream));
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+DSA_API dsa_status dsa_indexer_scores(const dsa_indexer_in* in, const int32_t* rows,
+                                      int32_t n_rows, float* scores, int64_t ld_scores,
+                                      int32_t n_cols, void* ws, size_t ws_bytes,
+                                      dsa_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  DSA_TRY(check_indexer(in));
+  if (scores == nullptr || n_rows < 1 || n_cols < 1 || ld_scores < n_cols)
+    return DSA_ERR_INVALID_ARG;
+  if (rows == nullptr && n_rows > in->n_q) return DSA_ERR_INVALID_ARG;
+  if (in->kv.kind == DSA_KV_PAGED && static_cast<int64_t>(n_cols) > int64_t(in->kv.max_pages) * kPage)
+    return DSA_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  DSA_TRY(device_info(&dev));
+  return run_indexer(*in, rows, 0, n_rows, scores, ld_scores, n_cols, 1, dev,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+DSA_API dsa_status dsa_topk(const float* scores, int64_t ld_scores, const int32_t* row_pos,
+                            int32_t n_rows, int32_t k, int32_t* idx, int64_t ld_idx,
+                            dsa_stream_t stream) {
+  if (scores == nullptr || row_pos == nullptr || idx == nullptr || n_rows < 1 || ld_scores < 1)
+    return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kKMax || ld_idx < k) return DSA_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  DSA_TRY(device_info(&dev));
+  return run_topk(scores, ld_scores, row_pos, 0, 0, n_rows, k, idx, ld_idx, dev,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+DSA_API dsa_status dsa_sparse_mqa_fwd(const dsa_attn_in* in, const int32_t* idx, int64_t ld_idx,
+                                      int32_t k, void* out, float* lse, void* ws,
+                                      size_t ws_bytes, dsa_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  DSA_TRY(check_attn(in));
+  if (idx == nullptr || out == nullptr || k < 1 || k > kKMax || ld_idx < k)
+    return DSA_ERR_INVALID_ARG;
+  if (in->dtype == DSA_BF16 && !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  DSA_TRY(device_info(&dev));
+  return run_attn(*in, idx, ld_idx, k, out, lse, dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+DSA_API dsa_status dsa_workspace_size(int32_t op, const dsa_indexer_in* indexer,
+                                      const dsa_attn_in* attn, int32_t n_rows, int32_t n_cols,
+                                      int32_t k, size_t* bytes) {
+  (void)attn;
+  (void)n_rows;
+  (void)n_cols;
+  if (bytes == nullptr) return DSA_ERR_INVALID_ARG;
+  *bytes = 0;
+  switch (op) {
+    case DSA_OP_INDEXER_SCORES:
+    case DSA_OP_TOPK:
+    case DSA_OP_SPARSE_MQA:
+      return DSA_OK;
+    case DSA_OP_FORWARD: {
+      DSA_TRY(check_indexer(indexer));
+      if (k < 1 || k > kKMax) return DSA_ERR_INVALID_ARG;
+      const ForwardPlan p = forward_plan(*indexer, k);
+      *bytes = p.scores_bytes + p.idx_bytes;
+      return DSA_OK;
+    }
+    default:
+      return DSA_ERR_INVALID_ARG;
+  }
+}
+
+DSA_API dsa_status dsa_forward(const dsa_indexer_in* indexer, const dsa_attn_in* attn,
+                               int32_t k, int32_t* idx_out, void* out, float* lse, void* ws,
+                               size_t ws_bytes, dsa_stream_t stream_) {
+  DSA_TRY(check_indexer(indexer));
+  DSA_TRY(check_attn(attn));
+  if (out == nullptr || k < 1 || k > kKMax) return DSA_ERR_INVALID_ARG;
+  if (indexer->n_q != attn->n_q || indexer->kv.kind != attn->kv_layout.kind)
+    return DSA_ERR_INVALID_ARG;
+  const bool paged = indexer->kv.kind == DSA_KV_PAGED;
+  if (!paged && indexer->n_keys != attn->n_keys) return DSA_ERR_INVALID_ARG;
+  if (paged && (indexer->kv.block_table != attn->kv_layout.block_table ||
+                indexer->kv.ctx_lens != attn->kv_layout.ctx_lens))
+    return DSA_ERR_INVALID_ARG;
+  const bool fp8 = indexer->dtype == DSA_E4M3 && attn->dtype == DSA_BF16;
+  const bool f32 = indexer->dtype == DSA_F32 && attn->dtype == DSA_F32;
+  if (!fp8 && !f32) return DSA_ERR_UNSUPPORTED;
+  if (attn->dtype == DSA_BF16 && !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  const ForwardPlan p = forward_plan(*indexer, k);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) ||
+      ws_bytes < p.scores_bytes + p.idx_bytes)
+    return DSA_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  DSA_TRY(device_info(&dev));
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  float* scores = static_cast<float*>(ws);
+  int32_t* idx = idx_out ? idx_out
+                         : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + p.scores_bytes);
+  const int32_t n_q = indexer->n_q;
+  if (paged) {
+    DSA_TRY(run_indexer(*indexer, nullptr, 0, n_q, scores, p.n_cols, p.n_cols, 0, dev, stream));
+    // query b sits at position ctx_lens[b] - 1
+    DSA_TRY(run_topk(scores, p.n_cols, indexer->kv.ctx_lens, 1, 0, n_q, k, idx, k, dev, stream));
+  } else {
+    const int32_t off = indexer->n_keys - n_q;  // position of query 0
+    for (int32_t q0 = 0; q0 < n_q; q0 += p.chunk) {
+      const int32_t rows = n_q - q0 < p.chunk ? n_q - q0 : p.chunk;
+      const int32_t cols = off + q0 + rows;    // keys any query of the block sees
+      DSA_TRY(run_indexer(*indexer, nullptr, q0, rows, scores, cols, cols, 0, dev, stream));
+      DSA_TRY(run_topk(scores, cols, nullptr, 0, off + q0, rows, k,
+                       idx + static_cast<int64_t>(q0) * k, k, dev, stream));
+    }
+  }
+  return run_attn(*attn, idx, k, k, out, lse, dev, stream);
+}
+
+DSA_API dsa_status dsa_check_status(dsa_stream_t stream) {
+  DeviceInfo* dev = nullptr;
+  DSA_TRY(device_info(&dev));
+  DSA_TRY_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  int v = 0;
+  DSA_TRY_CUDA(cudaMemcpyFromSymbol(&v, g_dsa_status, sizeof(int)));
+  if (v != 0) {
+    const int zero = 0;
+    DSA_TRY_CUDA(cudaMemcpyToSymbol(g_dsa_status, &zero, sizeof(int)));
+  }
+  return static_cast<dsa_status>(v);
+}
+
+DSA_API const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported dtype/dims/layout combination";
+    case DSA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small or misaligned";
+    case DSA_ERR_CUDA: return "CUDA runtime error";
+    case DSA_ERR_DEVICE_BOUNDS: return "device saw an index or page id out of range";
+    case DSA_ERR_TIMEOUT: return "a bounded device wait ran out";
+  }
+  return "unknown status";
+}
+
+DSA_API int32_t dsa_last_cuda_error(void) { return t_last_cuda_error; }
+
+DSA_API int32_t dsa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,293 @@
+// indexer_fp8.cu -- lightning-indexer scores on the 5th-generation tensor
+// cores (tcgen05, kind::f8f6f4) with the ReLU + weighted head reduction fused
+// into the TMEM epilogue.
+//
+// Definition (DeepSeek-V3.2-Exp report read-through on 53ai.com, section
+// "Innovative architecture: core design of DSA"; juhe.plus read-through, step 1
+// "Lightning Indexer"): for query token t and every preceding key s <= t,
+//     I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s]),
+// multi-head (j < 64), ReLU-gated, on FP8 inputs. With e4m3 codes and positive
+// per-token scales (q = sq[t] * code, k = sk[s] * code) this is
+//     I[t,s] = sk[s] * sum_j (w[t,j] * sq[t]) * ReLU(code_q[t,j] . code_k[s]),
+// which is what the kernel evaluates: the code dot products on the tensor core
+// (exact e4m3 products, f32 accumulation), then the epilogue below.
+//
+// Mapping: one MMA is D[128 keys, G*64] = K_tile[128 x 128 B] * Qgroup[G*64 x 128 B]^T
+// with keys on TMEM lanes and (query, head) on TMEM columns, so each epilogue
+// thread owns one key and reduces the 64 heads of a query inside its registers.
+//
+// Roles (192 threads, one CTA per SM, persistent over work units):
+//   warp 0    TMA producer: Q group (once per unit) and key tiles (6-stage ring)
+//   warp 1    TMEM owner and single-thread MMA issuer (2 accumulators in TMEM)
+//   warps 2-5 epilogue: tcgen05.ld -> ReLU * w -> head sum -> * sk -> global
+// A work unit is (group of G query rows, run of up to 16 key tiles of 128).
+#include "dsa_common.cuh"
+#include "dsa_kernels.h"
+#include "indexer_epilogue.cuh"
+
+namespace dsa {
+namespace {
+
+constexpr int kHeads = 64;
+constexpr int kDim = 128;  // e4m3 bytes per head row / per key row
+constexpr int kKeyTile = 128;
+constexpr int kMaxG = 4;
+constexpr int kStages = 6;
+constexpr int kTilesPerUnit = 16;
+constexpr int kThreads = 192;
+constexpr int kQBytes = kHeads * kDim;      // 8 KB per query
+constexpr int kKBytes = kKeyTile * kDim;    // 16 KB per key tile
+constexpr uint32_t kTmemCols = 512;
+
+struct __align__(1024) Smem {
+  uint8_t q[2][kMaxG * kQBytes];     // B operand (query group), double buffered per unit
+  uint8_t k[kStages][kKBytes];       // A operand (key tile) ring
+  float wq[kMaxG * kHeads];          // w[t,j] * sq[t] of the current unit
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t acc_full[2], acc_empty[2];
+  uint32_t tmem_base;
+};
+
+struct Unit {
+  int ng;             // query rows in the group
+  int row0;           // first row index
+  int qi[kMaxG];      // query indices
+  int pos[kMaxG];     // their positions (-1: invalid row, fully masked)
+  int max_pos;
+  int t0, t1;         // key-tile range of the unit
+  int t_end;          // tiles [t0, t_end) need an MMA (some query sees them)
+};
+
+__device__ __forceinline__ Unit get_unit(const IndexerFp8Args& a, int G, int n_chunks,
+                                         int n_tiles, int u, bool report_errors) {
+  Unit U;
+  const int g = u / n_chunks;
+  const int c = u - g * n_chunks;
+  U.row0 = g * G;
+  U.ng = min(G, a.qr.n_rows - U.row0);
+  U.max_pos = -1;
+#pragma unroll
+  for (int i = 0; i < kMaxG; ++i) {
+    U.qi[i] = 0;
+    U.pos[i] = -1;
+    if (i < U.ng) {
+      const int r = U.row0 + i;
+      int qi = a.qr.rows ? a.qr.rows[r] : a.qr.q_base + r;
+      int pos = -1;
+      if (qi < 0 || qi >= a.keys.n_q) {
+        if (report_errors) report(a.status, DSA_ERR_DEVICE_BOUNDS);
+        qi = 0;
+      } else if (a.keys.paged) {
+        const int ctx = a.keys.ctx_lens[qi];
+        if (ctx < 1 || ctx > a.keys.max_pages * 64) {
+          if (report_errors) report(a.status, DSA_ERR_DEVICE_BOUNDS);
+        } else {
+          pos = ctx - 1;
+        }
+      } else {
+        pos = a.keys.n_keys - a.keys.n_q + qi;
+      }
+      U.qi[i] = qi;
+      U.pos[i] = pos;
+      U.max_pos = max(U.max_pos, pos);
+    }
+  }
+  U.t0 = c * kTilesPerUnit;
+  U.t1 = min(n_tiles, U.t0 + kTilesPerUnit);
+  const int last = U.max_pos >= 0 ? U.max_pos / kKeyTile + 1 : 0;
+  U.t_end = max(U.t0, min(U.t1, last));
+  return U;
+}
+
+// Page id of logical page p of query qi, checked; 0 when out of range.
+__device__ __forceinline__ int page_of(const IndexerFp8Args& a, int qi, int p, bool report_errors) {
+  int page = a.keys.block_table[static_cast<int64_t>(qi) * a.keys.ld_block_table + p];
+  if (page < 0 || page >= a.keys.num_pages) {
+    if (report_errors) report(a.status, DSA_ERR_DEVICE_BOUNDS);
+    page = 0;
+  }
+  return page;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks, int n_tiles,
+                   int n_units) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                     ~uintptr_t(1023));
+  const int warp = warp_id();
+  const int lane = threadIdx.x & 31;
+  const int N = G * kHeads;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.q_full[i], 1);
+      mbar_init(&S.q_empty[i], 1);
+      mbar_init(&S.acc_full[i], 1);
+      mbar_init(&S.acc_empty[i], 128);
+    }
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&S.k_full[i], 1);
+      mbar_init(&S.k_empty[i], 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&a.map_q);
+    tma_prefetch_desc(&a.map_k);
+  }
+  if (warp == 1) tmem_alloc(&S.tmem_base, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = S.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0, ks = 0;
+      uint32_t kph = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
+        const Unit U = get_unit(a, G, n_chunks, n_tiles, u, true);
+        const int qb = it & 1;
+        const uint32_t qph = (it >> 1) & 1;
+        if (!mbar_wait(&S.q_empty[qb], qph ^ 1, a.status)) { ok = false; break; }
+        mbar_arrive_expect_tx(&S.q_full[qb], U.ng * kQBytes);
+        for (int i = 0; i < U.ng; ++i)
+          tma_load_3d(S.q[qb] + i * kQBytes, &a.map_q, 0, 0, U.qi[i], &S.q_full[qb]);
+        for (int t = U.t0; t < U.t_end; ++t) {
+          if (!mbar_wait(&S.k_empty[ks], kph ^ 1, a.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&S.k_full[ks], kKBytes);
+          if (!a.keys.paged) {
+            tma_load_2d(S.k[ks], &a.map_k, 0, t * kKeyTile, &S.k_full[ks]);
+          } else {
+            const int p0 = 2 * t;
+            const int pg0 = page_of(a, U.qi[0], p0, true);
+            const int pg1 = (p0 + 1) * 64 <= U.max_pos ? page_of(a, U.qi[0], p0 + 1, true) : pg0;
+            tma_load_2d(S.k[ks], &a.map_k, 0, pg0 * 64, &S.k_full[ks]);
+            tma_load_2d(S.k[ks] + kKBytes / 2, &a.map_k, 0, pg1 * 64, &S.k_full[ks]);
+          }
+          if (++ks == kStages) { ks = 0; kph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(static_cast<uint32_t>(N), 0, 0, 0, 0);
+      int it = 0, ks = 0, ab = 0;
+      uint32_t kph = 0, aph = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
+        const Unit U = get_unit(a, G, n_chunks, n_tiles, u, false);
+        const int qb = it & 1;
+        const uint32_t qph = (it >> 1) & 1;
+        if (!mbar_wait(&S.q_full[qb], qph, a.status)) break;
+        tc_fence_after();
+        const uint64_t bdesc = sw128_desc(smem_u32(S.q[qb]), 16, 1024);
+        for (int t = U.t0; t < U.t_end; ++t) {
+          if (!mbar_wait(&S.k_full[ks], kph, a.status) ||
+              !mbar_wait(&S.acc_empty[ab], aph ^ 1, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = sw128_desc(smem_u32(S.k[ks]), 16, 1024);
+          const uint32_t d = tmem_base + static_cast<uint32_t>(ab * N);
+#pragma unroll
+          for (int kk = 0; kk < kDim / 32; ++kk)
+            mma_f8(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+          mma_commit(&S.k_empty[ks]);
+          mma_commit(&S.acc_full[ab]);
+          if (++ks == kStages) { ks = 0; kph ^= 1; }
+          if (++ab == 2) { ab = 0; aph ^= 1; }
+        }
+        mma_commit(&S.q_empty[qb]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int sub = warp & 3;              // TMEM sub-partition of this warp
+    const int et = threadIdx.x - 64;       // 0..127
+    int ab = 0;
+    uint32_t aph = 0;
+    // After a timed-out wait the warp stops waiting and computing but keeps
+    // walking the same units, so every epilogue warp meets every named barrier.
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      const Unit U = get_unit(a, G, n_chunks, n_tiles, u, false);
+      named_bar_sync(1, 128);
+      for (int i = et; i < U.ng * kHeads; i += 128) {
+        const int g = i / kHeads;
+        const int qi = U.qi[g];
+        S.wq[i] = a.w[static_cast<int64_t>(qi) * a.ld_w + (i % kHeads)] * a.q_scale[qi];
+      }
+      named_bar_sync(1, 128);
+      for (int t = U.t0; t < U.t1 && ok; ++t) {
+        const int s = t * kKeyTile + sub * 32 + lane;
+        if (t >= U.t_end) {
+          if (a.write_masked && s < a.n_cols)
+            for (int g = 0; g < U.ng; ++g)
+              a.scores[static_cast<int64_t>(U.row0 + g) * a.ld_scores + s] = -INFINITY;
+          continue;
+        }
+        // key scale (0 for keys no query of the group sees)
+        float sk = 0.f;
+        if (s <= U.max_pos) {
+          if (!a.keys.paged) {
+            sk = a.k_scale[s];
+          } else {
+            const int pg = page_of(a, U.qi[0], s >> 6, false);
+            sk = a.k_scale[static_cast<int64_t>(pg) * 64 + (s & 63)];
+          }
+        }
+        if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tbase =
+            tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(ab * N);
+        for (int g = 0; g < U.ng; ++g) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tbase + g * kHeads, r0);
+          tmem_ld32(tbase + g * kHeads + 32, r1);
+          tmem_wait_ld();
+          const float score = indexer_score_from_dots(r0, r1, &S.wq[g * kHeads], sk);
+          if (s < a.n_cols)
+            a.scores[static_cast<int64_t>(U.row0 + g) * a.ld_scores + s] =
+                s <= U.pos[g] ? score : -INFINITY;
+        }
+        tc_fence_before();
+        mbar_arrive(&S.acc_empty[ab]);
+        if (++ab == 2) { ab = 0; aph ^= 1; }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_indexer_fp8(const IndexerFp8Args& a, int num_sms, cudaStream_t stream) {
+  const int G = a.keys.paged ? 1 : kMaxG;
+  const int n_groups = (a.qr.n_rows + G - 1) / G;
+  const int n_tiles = (a.n_cols + kKeyTile - 1) / kKeyTile;
+  const int n_chunks = (n_tiles + kTilesPerUnit - 1) / kTilesPerUnit;
+  const long long n_units_ll = static_cast<long long>(n_groups) * n_chunks;
+  if (n_units_ll <= 0) return cudaSuccess;
+  if (n_units_ll > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const int n_units = static_cast<int>(n_units_ll);
+  const size_t smem = sizeof(Smem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_fp8_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int grid = n_units < num_sms ? n_units : num_sms;
+  indexer_fp8_kernel<<<grid, kThreads, smem, stream>>>(a, G, n_chunks, n_tiles, n_units);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -157,11 +157,15 @@ def make_prefill(wl: Workload, device="cpu", seed: int = 0) -> PrefillInputs:
                          q, kv, None, needles)
 
 
-def make_decode(wl: Workload, device="cpu", seed: int = 0) -> DecodeInputs:
+def make_decode(wl: Workload, device="cpu", seed: int = 0, ctx_lens=None) -> DecodeInputs:
+    """ctx_lens (optional list) replaces the drawn context lengths."""
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     B = wl.B
     ctx = torch.randint(wl.ctx_min, wl.ctx_max + 1, (B,), generator=gen, device=device)
+    if ctx_lens is not None:
+        ctx = torch.tensor(ctx_lens, dtype=torch.int64, device=device)
+        B = len(ctx_lens)
     n_pages = (ctx + PAGE - 1) // PAGE
     num_pages = int(n_pages.sum().item())
     max_pages = (wl.ctx_max + PAGE - 1) // PAGE

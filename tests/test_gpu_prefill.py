@@ -1,0 +1,265 @@
+"""Parity of the FP8-indexer / bf16-attention prefill path (tensor-core
+kernels, called through the C ABI) against the oracle.
+
+Small cases cover every row and end in ragged tails (key tiles of 128, query
+groups of 4, key blocks of 64); the L=4096 workload is checked on every row for
+the indexer mask and the top-k, and on sampled rows for values; the 32K and
+128K workloads on sampled rows in the same launch configuration the benchmark
+times (dsa_forward)."""
+import dataclasses
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dsa_oracle as O
+from sparse_attention_long_tcgen05_b200.inputs import WORKLOADS, make_prefill, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def libs():
+    from sparse_attention_long_tcgen05_b200 import dsa
+    import dsa_testlib as T
+    return dsa, T
+
+
+def _wl(L, k=2048):
+    return dataclasses.replace(WORKLOADS[1], name=f"prefill_L{L}", L=L, k=k)
+
+
+def _scores(dsa, ind, rows_list, n_cols):
+    rows = torch.tensor(rows_list, dtype=torch.int32, device="cuda")
+    out = torch.empty(len(rows_list), n_cols, device="cuda")
+    dsa.dsa_indexer_scores(ind, rows, len(rows_list), out, n_cols)
+    assert dsa.dsa_check_status() == 0
+    return out
+
+
+@pytest.mark.parametrize("L", [1, 130, 777])
+def test_indexer_fp8_small_all_rows(libs, L):
+    dsa, T = libs
+    inp = make_prefill(_wl(L), device="cuda", seed=3)
+    ind, _ = T.prefill_structs(inp)
+    scores = torch.full((L, L + 5), 7.0, device="cuda")
+    dsa.dsa_indexer_scores(ind, None, L, scores, L)
+    assert dsa.dsa_check_status() == 0
+    g = scores.cpu().numpy()
+    assert np.all(g[:, L:] == 7.0), "wrote past n_cols"
+    rows = list(range(L))
+    qi, ki, w, _ = T.oracle_prefill_inputs(inp, rows)
+    ref = T.oracle_scores(qi, ki, w, rows, L)
+    T.assert_indexer_close(g[:, :L], ref)
+
+
+def test_indexer_fp8_query_suffix_positions(libs):
+    """n_q < n_keys: query i sits at position n_keys - n_q + i (chunked prefill)."""
+    dsa, T = libs
+    L, n_q = 1000, 300
+    inp = make_prefill(_wl(L), device="cuda", seed=4)
+    off = L - n_q
+    ind = dsa.indexer_in(inp.q_idx[off:], inp.k_idx, inp.w[off:], inp.q_scale[off:],
+                         inp.k_scale)
+    scores = torch.empty(n_q, L, device="cuda")
+    dsa.dsa_indexer_scores(ind, None, n_q, scores, L)
+    assert dsa.dsa_check_status() == 0
+    rows = list(range(off, L))
+    qi, ki, w, _ = T.oracle_prefill_inputs(inp, rows)
+    ref = T.oracle_scores(qi, ki, w, rows, L)
+    T.assert_indexer_close(scores.cpu().numpy(), ref)
+
+
+def test_indexer_rows_subset_bitexact_with_all_rows(libs):
+    """Scores for an arbitrary row subset equal the all-rows scores bit for bit
+    (rows are grouped 4 to an MMA in any order)."""
+    dsa, T = libs
+    L = 1100
+    inp = make_prefill(_wl(L), device="cuda", seed=5)
+    ind, _ = T.prefill_structs(inp)
+    full = torch.empty(L, L, device="cuda")
+    dsa.dsa_indexer_scores(ind, None, L, full, L)
+    rows = [1099, 3, 640, 641, 0, 17, 1000]
+    sub = _scores(dsa, ind, rows, L)
+    assert torch.equal(sub, full[torch.tensor(rows, device="cuda")])
+
+
+def test_topk_bitexact_L4096_all_rows(libs):
+    dsa, T = libs
+    inp = make_prefill(WORKLOADS[1], device="cuda", seed=0)
+    L, k = inp.wl.L, inp.wl.k
+    ind, _ = T.prefill_structs(inp)
+    scores = torch.empty(L, L, device="cuda")
+    dsa.dsa_indexer_scores(ind, None, L, scores, L)
+    idx = torch.empty(L, k, dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(scores, torch.arange(L, dtype=torch.int32, device="cuda"), k, idx)
+    assert dsa.dsa_check_status() == 0
+    ref = T.topk_oracle_on(scores.double().cpu().numpy(), np.arange(L), k)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+
+
+def test_topk_ties_and_signed_zero(libs):
+    dsa, T = libs
+    rng = np.random.default_rng(1)
+    R, n = 37, 5000
+    pool = np.array([-1.0, -0.0, 0.0, 0.25, 2.0, -np.inf, np.nan], dtype=np.float32)
+    s = rng.choice(pool, size=(R, n)).astype(np.float32)
+    s[5] = 0.0
+    s[6] = -0.0
+    s[7] = rng.standard_normal(n).astype(np.float32)
+    pos = rng.integers(0, n, R).astype(np.int32)
+    pos[:3] = [0, 2047, n - 1]
+    for k in (1, 7, 2048):
+        idx = torch.empty(R, k, dtype=torch.int32, device="cuda")
+        dsa.dsa_topk(torch.from_numpy(s).cuda(), torch.from_numpy(pos).cuda(), k, idx)
+        assert dsa.dsa_check_status() == 0
+        ref = T.topk_oracle_on(s.astype(np.float64), pos, k)
+        assert np.array_equal(idx.cpu().numpy(), ref), k
+
+
+def _attention_case(dsa, T, L, k, seed, rows=None):
+    inp = make_prefill(_wl(L, k), device="cuda", seed=seed)
+    rng = np.random.default_rng(seed)
+    idx_h = T.topk_oracle_on(rng.standard_normal((L, L)), np.arange(L), k)
+    idx = torch.from_numpy(idx_h).cuda()
+    _, att = T.prefill_structs(inp)
+    out = torch.empty(L, 128, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(L, 128, device="cuda")
+    dsa.dsa_sparse_mqa_fwd(att, idx, k, out, lse)
+    assert dsa.dsa_check_status() == 0
+    rows = list(range(L)) if rows is None else rows
+    q = inp.q[torch.tensor(rows, device="cuda")].double().cpu().numpy()
+    kv_sub, idx_local = T.gather_kv_rows(inp.kv, idx_h[rows])
+    o_ref, l_ref = O.sparse_mqa(q, kv_sub, None, idx_local, list(range(len(rows))),
+                                inp.wl.scale, 512)
+    r = torch.tensor(rows, device="cuda")
+    return T.assert_attention_close(out[r].float().cpu().numpy(), lse[r].cpu().numpy(), o_ref,
+                                    l_ref)
+
+
+def test_attention_bf16_dense_prefix(libs):
+    """k >= L: every row attends to its whole prefix (one to five 64-key blocks,
+    the last one ragged)."""
+    dsa, T = libs
+    _attention_case(dsa, T, L=300, k=2048, seed=6)
+
+
+def test_attention_bf16_ragged_k(libs):
+    dsa, T = libs
+    _attention_case(dsa, T, L=1000, k=300, seed=7)
+
+
+def test_attention_bf16_L4096_sampled(libs):
+    dsa, T = libs
+    rows = sample_rows(4096, 96, seed=1)
+    _attention_case(dsa, T, L=4096, k=2048, seed=0, rows=rows)
+
+
+def test_attention_single_key_rows(libs):
+    """Rows whose selection is one key output that key's value row (softmax of
+    one logit is 1)."""
+    dsa, T = libs
+    L = 200
+    inp = make_prefill(_wl(L), device="cuda", seed=8)
+    k = 64
+    idx = torch.full((L, k), -1, dtype=torch.int32, device="cuda")
+    sel = torch.randint(0, L, (L,), device="cuda")
+    sel = torch.minimum(sel, torch.arange(L, device="cuda"))
+    ar = torch.arange(L, device="cuda")
+    idx[ar, (ar * 7) % k] = sel.int()
+    _, att = T.prefill_structs(inp)
+    out = torch.empty(L, 128, 512, dtype=torch.bfloat16, device="cuda")
+    dsa.dsa_sparse_mqa_fwd(att, idx, k, out, None)
+    assert dsa.dsa_check_status() == 0
+    want = inp.kv[sel.long(), :512][:, None, :].expand(L, 128, 512)
+    assert torch.equal(out, want)
+
+
+def _forward(dsa, T, inp):
+    wl = inp.wl
+    L, k = wl.L, wl.k
+    ind, att = T.prefill_structs(inp)
+    ws = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_FORWARD, ind, att, 0, 0, k))
+    idx = torch.empty(L, k, dtype=torch.int32, device="cuda")
+    out = torch.empty(L, 128, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(L, 128, device="cuda")
+    dsa.dsa_forward(ind, att, k, idx, out, lse, ws)
+    assert dsa.dsa_check_status() == 0
+    return ind, att, idx, out, lse
+
+
+def _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, rows):
+    wl = inp.wl
+    L, k = wl.L, wl.k
+    # indexer values on the sampled rows
+    sc = _scores(dsa, ind, rows, L)
+    qi, ki, w, q = T.oracle_prefill_inputs(inp, rows)
+    ref_scores = T.oracle_scores(qi, ki, w, rows, L)
+    T.assert_indexer_close(sc.cpu().numpy(), ref_scores)
+    # the fused selection equals top-k of the standalone scores, bit for bit,
+    # and equals the oracle's top-k of those same scores
+    r = torch.tensor(rows, device="cuda")
+    g_idx = idx[r].cpu().numpy()
+    ref_idx = T.topk_oracle_on(sc.double().cpu().numpy(), np.array(rows), k)
+    assert np.array_equal(g_idx, ref_idx)
+    # attention on the sampled rows with those indices
+    kv_sub, idx_local = T.gather_kv_rows(inp.kv, g_idx)
+    o_ref, l_ref = O.sparse_mqa(q, kv_sub, None, idx_local, list(range(len(rows))), wl.scale,
+                                512)
+    T.assert_attention_close(out[r].float().cpu().numpy(), lse[r].cpu().numpy(), o_ref, l_ref)
+    # diagnostic: overlap with the oracle's own selection (its own scores)
+    own = T.topk_oracle_on(ref_scores, np.array(rows), k)
+    overlap = np.mean([len(set(a[a >= 0]) & set(b[b >= 0])) / max(1, (b >= 0).sum())
+                       for a, b in zip(g_idx, own)])
+    assert overlap > 0.95, overlap
+
+
+def test_forward_L4096(libs):
+    dsa, T = libs
+    inp = make_prefill(WORKLOADS[1], device="cuda", seed=0)
+    ind, att, idx, out, lse = _forward(dsa, T, inp)
+    L, k = inp.wl.L, inp.wl.k
+    # every row: the fused selection is the standalone top-k of standalone scores
+    scores = torch.empty(L, L, device="cuda")
+    dsa.dsa_indexer_scores(ind, None, L, scores, L)
+    idx_s = torch.empty(L, k, dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(scores, torch.arange(L, dtype=torch.int32, device="cuda"), k, idx_s)
+    assert torch.equal(idx, idx_s)
+    out_s = torch.empty_like(out)
+    lse_s = torch.empty_like(lse)
+    dsa.dsa_sparse_mqa_fwd(att, idx_s, k, out_s, lse_s)
+    assert torch.equal(out, out_s) and torch.equal(lse, lse_s)
+    # structure of the selection: causal, ascending, min(k, t+1) entries
+    ih = idx.cpu().numpy()
+    cnt = (ih >= 0).sum(1)
+    assert np.array_equal(cnt, np.minimum(k, np.arange(L) + 1))
+    assert np.all(ih.max(1) <= np.arange(L))
+    _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, sample_rows(L, 64, seed=1))
+
+
+def test_forward_L32768_needles(libs):
+    dsa, T = libs
+    inp = make_prefill(WORKLOADS[2], device="cuda", seed=0)
+    ind, att, idx, out, lse = _forward(dsa, T, inp)
+    rows = sample_rows(inp.wl.L, 48, seed=1)
+    _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, rows)
+    # the planted x3 keys are over-represented in the selections of long rows
+    needles = set(inp.needles.cpu().tolist())
+    ih = idx.cpu().numpy()
+    long_rows = [t for t in rows if t >= 8192]
+    frac = np.mean([np.isin(ih[t][ih[t] >= 0], list(needles)).mean() for t in long_rows])
+    base = 64 / 4096
+    assert frac > 4 * base, frac
+
+
+@pytest.mark.skipif(os.environ.get("DSA_SKIP_128K") == "1", reason="DSA_SKIP_128K=1")
+def test_forward_L131072_sampled(libs):
+    dsa, T = libs
+    inp = make_prefill(WORKLOADS[3], device="cuda", seed=0)
+    ind, att, idx, out, lse = _forward(dsa, T, inp)
+    n = int(os.environ.get("DSA_128K_ROWS", "32"))
+    rows = sample_rows(inp.wl.L, n, seed=1)
+    _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, rows)
+    ih = idx[torch.tensor(rows, device="cuda")].cpu().numpy()
+    assert np.array_equal((ih >= 0).sum(1), np.minimum(2048, np.array(rows) + 1))

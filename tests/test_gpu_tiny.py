@@ -1,0 +1,123 @@
+"""Parity of the float32 path on the tiny workload (L=256, H_I=4, d_I=32,
+8 heads, d=64, separate V, k=64) against the oracle, every row."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dsa_oracle as O
+from sparse_attention_long_tcgen05_b200.inputs import WORKLOADS, make_prefill
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def env():
+    from sparse_attention_long_tcgen05_b200 import dsa
+    import dsa_testlib as T
+    inp = make_prefill(WORKLOADS[0], device="cuda", seed=0)
+    return dsa, T, inp
+
+
+def _host(t):
+    return t.double().cpu().numpy()
+
+
+def test_tiny_indexer(env):
+    dsa, T, inp = env
+    L = inp.wl.L
+    ind, _ = T.prefill_structs(inp)
+    scores = torch.empty(L, L, device="cuda")
+    dsa.dsa_indexer_scores(ind, None, L, scores, L)
+    assert dsa.dsa_check_status() == 0
+    ref = O.indexer_scores(_host(inp.q_idx), _host(inp.k_idx), _host(inp.w), list(range(L)),
+                           list(range(L)), L)
+    T.assert_indexer_close(scores.cpu().numpy(), ref, rel=1e-5, floor=1e-3)
+    # w ~ U(0,1) >= 0: every visible score is >= 0 (ReLU gating)
+    s = scores.cpu().numpy()
+    assert np.all(s[np.isfinite(s)] >= 0)
+
+
+def test_tiny_topk_bitexact(env):
+    dsa, T, inp = env
+    L, k = inp.wl.L, inp.wl.k
+    ind, _ = T.prefill_structs(inp)
+    scores = torch.empty(L, L, device="cuda")
+    dsa.dsa_indexer_scores(ind, None, L, scores, L)
+    pos = torch.arange(L, dtype=torch.int32, device="cuda")
+    idx = torch.empty(L, k, dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(scores, pos, k, idx)
+    assert dsa.dsa_check_status() == 0
+    ref = T.topk_oracle_on(scores.double().cpu().numpy(), np.arange(L), k)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+
+
+def test_tiny_attention(env):
+    dsa, T, inp = env
+    wl = inp.wl
+    L, k = wl.L, wl.k
+    rng = np.random.default_rng(0)
+    idx_h = T.topk_oracle_on(rng.standard_normal((L, L)), np.arange(L), k)
+    idx = torch.from_numpy(idx_h).cuda()
+    _, att = T.prefill_structs(inp)
+    out = torch.empty(L, wl.H, wl.D_V, device="cuda")
+    lse = torch.empty(L, wl.H, device="cuda")
+    dsa.dsa_sparse_mqa_fwd(att, idx, k, out, lse)
+    assert dsa.dsa_check_status() == 0
+    o_ref, l_ref = O.sparse_mqa(_host(inp.q), _host(inp.kv), _host(inp.v), idx_h, list(range(L)),
+                                wl.scale, wl.D_V)
+    T.assert_attention_close(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, max_abs=1e-4,
+                             rel_rms=1e-5, lse_abs=1e-4)
+
+
+def test_tiny_sparse_equals_dense_when_k_covers_prefix(env):
+    """k >= t+1 for every row: DSA reduces to dense causal attention."""
+    dsa, T, inp = env
+    wl = inp.wl
+    L = wl.L
+    k = L
+    idx = torch.empty(L, k, dtype=torch.int32, device="cuda")
+    scores = torch.zeros(L, L, device="cuda")
+    dsa.dsa_topk(scores, torch.arange(L, dtype=torch.int32, device="cuda"), k, idx)
+    _, att = T.prefill_structs(inp)
+    out = torch.empty(L, wl.H, wl.D_V, device="cuda")
+    lse = torch.empty(L, wl.H, device="cuda")
+    dsa.dsa_sparse_mqa_fwd(att, idx, k, out, lse)
+    assert dsa.dsa_check_status() == 0
+    o_ref, l_ref = O.dense_causal_attention(_host(inp.q), _host(inp.kv), _host(inp.v), wl.scale)
+    T.assert_attention_close(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, max_abs=1e-4,
+                             rel_rms=1e-5, lse_abs=1e-4)
+
+
+def test_tiny_forward_matches_steps_and_oracle(env):
+    dsa, T, inp = env
+    wl = inp.wl
+    L, k = wl.L, wl.k
+    ind, att = T.prefill_structs(inp)
+    ws = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_FORWARD, ind, att, 0, 0, k))
+    idx_f = torch.empty(L, k, dtype=torch.int32, device="cuda")
+    out_f = torch.empty(L, wl.H, wl.D_V, device="cuda")
+    lse_f = torch.empty(L, wl.H, device="cuda")
+    dsa.dsa_forward(ind, att, k, idx_f, out_f, lse_f, ws)
+    assert dsa.dsa_check_status() == 0
+    # step by step through the ABI
+    scores = torch.empty(L, L, device="cuda")
+    dsa.dsa_indexer_scores(ind, None, L, scores, L)
+    idx_s = torch.empty(L, k, dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(scores, torch.arange(L, dtype=torch.int32, device="cuda"), k, idx_s)
+    out_s = torch.empty_like(out_f)
+    lse_s = torch.empty_like(lse_f)
+    dsa.dsa_sparse_mqa_fwd(att, idx_s, k, out_s, lse_s)
+    assert torch.equal(idx_f, idx_s)
+    assert torch.equal(out_f, out_s) and torch.equal(lse_f, lse_s)
+    # whole forward in the oracle (its own scores and selection)
+    sc, idx_o, o_ref, l_ref = O.forward_prefill_rows(
+        _host(inp.q_idx), _host(inp.k_idx), _host(inp.w), _host(inp.q), _host(inp.kv),
+        _host(inp.v), list(range(L)), k, wl.scale, wl.D_V)
+    agree = np.mean([len(set(a[a >= 0]) & set(b[b >= 0])) / max(1, (b >= 0).sum())
+                     for a, b in zip(idx_f.cpu().numpy(), idx_o)])
+    assert agree > 0.99
+    same = np.all(idx_f.cpu().numpy() == idx_o, axis=1)
+    T.assert_attention_close(out_f.cpu().numpy()[same], lse_f.cpu().numpy()[same], o_ref[same],
+                             l_ref[same], max_abs=1e-4, rel_rms=1e-5, lse_abs=1e-4)
