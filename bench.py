@@ -1,0 +1,497 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA forward path on B200: 128K-token prefill tokens/s
+(headline) and batch-64 paged decode tokens/s, each with its roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1). The path has no cross-GPU exchange:
+each rank runs its own full workload (independent sequences), so scaling is
+weak and `value` is the tokens of all ranks divided by the slowest rank's time.
+Rank 0 prints one JSON line.
+
+A prefill step is one dsa_forward over L=131072 tokens (indexer -> top-k ->
+sparse attention) with every input already resident in HBM; the inputs are far
+larger than L2 (q alone is 19.3 GB). A decode step is one dsa_forward over 64
+sequences; L2 is flushed before every decode step, outside the timed events.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DSA prefill tokens/s at 128K and decode tokens/s (1 B200) + % of roofline"
+
+DECODE_WL = 4
+
+
+# ----------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"],
+                "bf16_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_traffic(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None
+    when the kernel's source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, "sparse_attention_long_tcgen05_b200", "csrc", d["source"])
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return d["bytes_per_launch"] if sha == d.get("source_sha") else None
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons while timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append(parts)
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        loaded = [r for r in rows if (num(r[4]) or 0) >= 50] or rows
+        sm = [num(r[1]) for r in loaded if num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(4)
+                          if r[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(loaded[0][2]), "reasons": reasons,
+                "samples_under_load": len(loaded),
+                "power_w_max": max((num(r[3]) or 0) for r in loaded)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(fn, steps, warmup, world, pre=None):
+    """Average ms per call of fn() over `steps` calls, CUDA events on the
+    current stream, warm-up first, barrier + synchronize on both sides, max
+    over ranks. `pre` (untimed) runs before every call when given."""
+    for _ in range(warmup):
+        if pre:
+            pre()
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    if pre is None:
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+    else:
+        total = 0.0
+        for _ in range(steps):
+            pre()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            total += a.elapsed_time(b)
+        ms = total / steps
+    barrier(world)
+    torch.cuda.synchronize()
+    return max_over_ranks(ms, world)
+
+
+def pinned_copy(t: torch.Tensor) -> torch.Tensor:
+    h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    h.copy_(t)
+    return h
+
+
+def attention_pairs(L, k):
+    """Selected (query, key) pairs of a causal prefill: sum_t min(k, t+1)."""
+    m = min(k, L)
+    return m * (m + 1) // 2 + (L - m) * k
+
+
+# ----------------------------------------------------------------- our arm
+
+def run_ours(args, world, rank, local):
+    from sparse_attention_long_tcgen05_b200 import _build
+    if rank == 0 or not os.path.exists(_build.LIB):
+        _build.build()
+    barrier(world)
+    from sparse_attention_long_tcgen05_b200 import dsa
+    from sparse_attention_long_tcgen05_b200.inputs import WORKLOADS, make_prefill, make_decode
+
+    peaks = load_peaks()
+    fp8_sustained = 2.0 * peaks["bf16_sustained"]   # FP8 dense = 2x bf16 (nominal ratio)
+    wl = next(w for w in WORKLOADS.values() if w.name == args.workload)
+    L, k = wl.L, wl.k
+    inp = make_prefill(wl, device="cuda", seed=rank)
+    ind = dsa.indexer_in(inp.q_idx, inp.k_idx, inp.w, inp.q_scale, inp.k_scale)
+    att = dsa.attn_in(inp.q, inp.kv, wl.scale, wl.D_V)
+    ws = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_FORWARD, ind, att, 0, 0, k))
+    idx = torch.empty(L, k, dtype=torch.int32, device="cuda")
+    out = torch.empty(L, wl.H, wl.D_V, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(L, wl.H, device="cuda")
+
+    def fwd():
+        dsa.dsa_forward(ind, att, k, idx, out, lse, ws)
+
+    def sel():
+        dsa.dsa_select(ind, k, idx, ws)
+
+    def attn():
+        dsa.dsa_sparse_mqa_fwd(att, idx, k, out, lse)
+
+    with Clocks(local) as clk:
+        n0 = dsa.dsa_launch_counter()
+        ms = timed(fwd, args.steps, args.warmup, world)
+        launches = dsa.dsa_launch_counter() - n0
+    st = dsa.dsa_check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {dsa.status_string(st)}")
+    # launches counted above include the warm-up calls: scale to the timed ones
+    per_call = launches / (args.steps + args.warmup)
+    ms_sel = timed(sel, args.steps, 1, world)
+    ms_attn = timed(attn, args.steps, 1, world)
+
+    idx_flops = 2.0 * wl.H_I * wl.d_I * (L * (L + 1) / 2)
+    attn_flops = 2.0 * wl.H * (wl.D_K + wl.D_V) * attention_pairs(L, k)
+    sel_tf = idx_flops / (ms_sel * 1e-3) / 1e12
+    attn_tf = attn_flops / (ms_attn * 1e-3) / 1e12
+    stages = {
+        "select_ms": ms_sel, "select_fp8_tflops": sel_tf,
+        "select_frac_fp8_sustained": sel_tf / fp8_sustained,
+        "attention_ms": ms_attn, "attention_bf16_tflops": attn_tf,
+        "attention_frac_bf16_sustained": attn_tf / peaks["bf16_sustained"],
+        "indexer_flops": idx_flops, "attention_flops": attn_flops,
+    }
+    if ms_sel >= ms_attn:
+        roof = {"kernel": "indexer_fp8_kernel+topk_kernel (dsa_select)", "bound": "tensor",
+                "achieved": sel_tf, "peak": fp8_sustained, "unit": "TFLOP/s",
+                "frac": sel_tf / fp8_sustained,
+                "peak_note": f"FP8 dense = 2 x measured bf16 sustained ({peaks['source']})",
+                "traffic": kernel_traffic("indexer_fp8_kernel")}
+    else:
+        roof = {"kernel": "sparse_mqa_bf16_kernel", "bound": "tensor", "achieved": attn_tf,
+                "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                "frac": attn_tf / peaks["bf16_sustained"],
+                "peak_note": f"bf16 dense sustained ({peaks['source']})",
+                "traffic": kernel_traffic("sparse_mqa_bf16_kernel")}
+
+    # ------------------------------------------------------------ e2e (host buffers)
+    e2e = None
+    if not args.skip_e2e:
+        try:
+            e2e = prefill_e2e(dsa, inp, ind, att, ws, idx, out, lse, k, args, world)
+        except Exception as ex:  # pinned-memory limits on the host
+            e2e = {"value": None, "unit": "tokens/s", "error": str(ex)[:200]}
+
+    # ------------------------------------------------------------ cpu baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        cpu = oracle_prefill_rate(inp, wl, budget_s=args.cpu_budget)
+
+    value_tok = world * L / (ms * 1e-3)
+    res = {
+        "metric": METRIC, "value": value_tok, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3+bf16 (f32 accumulate)", "data": "synthetic",
+        "config": {"workload": wl.name, "L": L, "k": k, "H_I": wl.H_I, "d_I": wl.d_I,
+                   "H": wl.H, "d_qk": wl.D_K, "d_v": wl.D_V, "seed": "rank",
+                   "l2": "inputs larger than L2 (q alone 19.3 GB)",
+                   "parallelism": f"replicas x{world} (independent sequences)"},
+        "roofline": roof, "stages": stages, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": int(round(per_call * args.steps)),
+        "clocks": clk.summary(),
+    }
+    del inp, out, idx, lse, ws
+    torch.cuda.empty_cache()
+    if not args.skip_decode:
+        res["decode"] = run_decode(args, world, rank, local, peaks, dsa, make_decode,
+                                   WORKLOADS[DECODE_WL])
+    return res
+
+
+def prefill_e2e(dsa, inp, ind, att, ws, idx, out, lse, k, args, world):
+    """Same metric through the public call with host buffers: every step copies
+    its inputs from pinned host memory and reads the attention output back."""
+    dev_in = [inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.q, inp.kv]
+    host_in = [pinned_copy(t) for t in dev_in]
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def step():
+        for h, d in zip(host_in, dev_in):
+            d.copy_(h, non_blocking=True)
+        dsa.dsa_forward(ind, att, k, idx, out, lse, ws)
+        host_out.copy_(out, non_blocking=True)
+        host_lse.copy_(lse, non_blocking=True)
+
+    ms = timed(step, args.e2e_steps, 1, world)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * 4
+    return {"value": world * inp.wl.L / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "steps": args.e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def oracle_prefill_rate(inp, wl, budget_s=15.0, rows_cap=None):
+    """The CPU oracle as it stands on a bounded sample of query rows of the same
+    workload (uniform rows, so the mean prefix is ~L/2): tokens/s = rows/wall."""
+    import numpy as np
+    from oracle import dsa_oracle as O
+    from sparse_attention_long_tcgen05_b200.inputs import sample_rows
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((p.get("num_threads") or 0) for p in threadpool_info()) or os.cpu_count()
+    except Exception:
+        cores = os.cpu_count()
+    rows = sample_rows(wl.L, 512, seed=1)
+    rng = np.random.default_rng(2)
+    rng.shuffle(rows)
+    k_deq = O.dequantize(inp.k_idx.cpu().numpy(), inp.k_scale.cpu().numpy())
+    kv = inp.kv.cpu()
+    done = 0
+    t0 = time.time()
+    for t in rows:
+        if time.time() - t0 > budget_s or (rows_cap and done >= rows_cap):
+            break
+        q_deq = O.dequantize(inp.q_idx[t].cpu().numpy()[None], inp.q_scale[t:t + 1].cpu().numpy())
+        sc = O.indexer_row(q_deq[0], k_deq[: t + 1], inp.w[t].double().cpu().numpy())
+        sel = O.topk_row(sc, t, wl.k)
+        sel = sel[sel >= 0]
+        keys = kv[torch.from_numpy(sel).long()].double().numpy()
+        O.attend(inp.q[t].double().cpu().numpy(), keys, keys[:, : wl.D_V], wl.scale)
+        done += 1
+    wall = time.time() - t0
+    return {"value": done / wall, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} uniformly drawn query rows of {wl.name} "
+                      f"(indexer+top-k+attention per row, float64), {wall:.1f} s wall"}
+
+
+def run_decode(args, world, rank, local, peaks, dsa, make_decode, wl):
+    inp = make_decode(wl, device="cuda", seed=rank)
+    lay = dsa.paged_layout(inp.block_table, inp.ctx_lens, inp.num_pages)
+    ind = dsa.indexer_in(inp.q_idx, inp.k_cache, inp.w, inp.q_scale, inp.k_cache_scale.view(-1),
+                         kv=lay)
+    att = dsa.attn_in(inp.q, inp.kv_cache, wl.scale, wl.D_V, kv_layout=lay)
+    B, k = inp.q.shape[0], wl.k
+    ws = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_FORWARD, ind, att, 0, 0, k))
+    idx = torch.empty(B, k, dtype=torch.int32, device="cuda")
+    out = torch.empty(B, wl.H, wl.D_V, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, wl.H, device="cuda")
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    flush_buf = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device="cuda")
+
+    def flush():
+        flush_buf.fill_(1.0)
+
+    def fwd():
+        dsa.dsa_forward(ind, att, k, idx, out, lse, ws)
+
+    def sel():
+        dsa.dsa_select(ind, k, idx, ws)
+
+    def attn():
+        dsa.dsa_sparse_mqa_fwd(att, idx, k, out, lse)
+
+    steps = max(args.steps, 10)
+    ms = timed(fwd, steps, args.warmup, world, pre=flush)
+    ms_sel = timed(sel, steps, 1, world, pre=flush)
+    ms_attn = timed(attn, steps, 1, world, pre=flush)
+    ctx = inp.ctx_lens.long()
+    n_sel = torch.clamp(ctx, max=k)
+    scan_bytes = float((ctx * (wl.d_I + 4)).sum())
+    gather_bytes = float((n_sel * wl.D_K * 2).sum())
+    qo_bytes = B * (wl.H * wl.D_K * 2 + wl.H * wl.D_V * 2 + wl.H * 4 + wl.H_I * wl.d_I +
+                    wl.H_I * 4 + 4)
+    step_bytes = scan_bytes + gather_bytes + qo_bytes
+    hbm = peaks["hbm_gbs"]
+    sel_gbs = (scan_bytes + B * (wl.H_I * wl.d_I + wl.H_I * 4)) / (ms_sel * 1e-3) / 1e9
+    attn_gbs = (gather_bytes + B * (wl.H * wl.D_K * 2 + wl.H * wl.D_V * 2)) / (ms_attn * 1e-3) / 1e9
+    step_gbs = step_bytes / (ms * 1e-3) / 1e9
+    # e2e: the caches stay resident; per step the new query tensors go up and
+    # the attention output comes back
+    e2e = None
+    if not args.skip_e2e:
+        dev_in = [inp.q_idx, inp.q_scale, inp.w, inp.q, inp.ctx_lens, inp.block_table]
+        host_in = [pinned_copy(t) for t in dev_in]
+        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def step():
+            for h, d in zip(host_in, dev_in):
+                d.copy_(h, non_blocking=True)
+            fwd()
+            host_out.copy_(out, non_blocking=True)
+        ms_e2e = timed(step, steps, 1, world, pre=flush)
+        e2e = {"value": world * B / (ms_e2e * 1e-3), "unit": "tokens/s", "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host_in),
+               "d2h_bytes_per_step": host_out.numel() * host_out.element_size()}
+    return {
+        "workload": wl.name, "value": world * B / (ms * 1e-3), "unit": "tokens/s",
+        "ms_per_step": ms, "steps": steps, "l2": "flushed before every step (untimed)",
+        "mean_ctx": float(ctx.float().mean()),
+        "roofline": {"kernel": "whole decode step", "bound": "hbm", "achieved": step_gbs,
+                     "peak": hbm, "unit": "GB/s", "frac": step_gbs / hbm,
+                     "algorithmic_bytes_per_step": step_bytes, "traffic": None},
+        "stages": {"select_ms": ms_sel, "select_gbs": sel_gbs, "select_frac_hbm": sel_gbs / hbm,
+                   "attention_ms": ms_attn, "attention_gbs": attn_gbs,
+                   "attention_frac_hbm": attn_gbs / hbm},
+        "e2e": e2e,
+    }
+
+
+# ----------------------------------------------------------------- reference arm
+
+def run_reference(args, world, rank):
+    """The oracle as it stands on the host cores: each step is a bounded sample
+    of query rows of the same workload; tokens/s = rows / wall time."""
+    from sparse_attention_long_tcgen05_b200.inputs import WORKLOADS, make_prefill
+    wl = next(w for w in WORKLOADS.values() if w.name == args.workload)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_prefill(wl, device=dev, seed=0)   # input generation only, untimed
+    rates = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_prefill_rate(inp, wl, budget_s=args.ref_step_s)
+        if i >= args.warmup:
+            rates.append(r)
+    value = statistics.mean(r["value"] for r in rates)
+    cpu = dict(rates[-1])
+    cpu["value"] = value
+    cpu["sample"] = (f"{args.steps} steps of ~{args.ref_step_s:.0f} s, each "
+                     + rates[-1]["sample"])
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "L": wl.L, "k": wl.k},
+            "cpu_baseline": cpu,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_L131072",
+                    choices=["prefill_L4096", "prefill_L32768_needle", "prefill_L131072"],
+                    help="prefill workload of the headline line (smaller ones for profiling)")
+    ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-step-s", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup() if torch.cuda.is_available() else (1, 0, 0)
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        res = run_reference(args, world, rank)
+    else:
+        res = run_ours(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -135,7 +135,8 @@ typedef enum dsa_op {
   DSA_OP_INDEXER_SCORES = 0,
   DSA_OP_TOPK = 1,
   DSA_OP_SPARSE_MQA = 2,
-  DSA_OP_FORWARD = 3
+  DSA_OP_FORWARD = 3,
+  DSA_OP_SELECT = 4
 } dsa_op;
 
 /* Step 1 alone: lightning-indexer scores for selected query rows.
@@ -171,6 +172,14 @@ DSA_API dsa_status dsa_sparse_mqa_fwd(const dsa_attn_in* in, const int32_t* idx,
                                       int32_t k, void* out, float* lse, void* ws,
                                       size_t ws_bytes, dsa_stream_t stream);
 
+/* Steps 1-2 fused: the selection alone (indexer -> top-k), streamed over
+ * bounded blocks of queries so the n_q x n_keys score matrix never exists.
+ * idx: [n_q, ld_idx] int32 (ld_idx >= k), same contents and rules as
+ * dsa_topk(dsa_indexer_scores(...)) bit for bit.
+ * Workspace: dsa_workspace_size(DSA_OP_SELECT). */
+DSA_API dsa_status dsa_select(const dsa_indexer_in* indexer, int32_t k, int32_t* idx,
+                              int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
 /* Steps 1-3 fused: indexer -> top-k -> sparse attention without ever holding
  * the n_q x n_keys score matrix (prefill streams the indexer over bounded
  * blocks of queries). idx_out (nullable, [n_q, k] int32) receives the
@@ -195,6 +204,10 @@ DSA_API const char* dsa_status_string(dsa_status status);
 
 /* The cudaError_t value behind the last DSA_ERR_CUDA on this thread (0 if none). */
 DSA_API int32_t dsa_last_cuda_error(void);
+
+/* Number of kernel launches this process has issued through the library so
+ * far (all devices, all threads). Lets a caller count launches in a region. */
+DSA_API int64_t dsa_launch_counter(void);
 
 /* Library version, major*10000 + minor*100 + patch. */
 DSA_API int32_t dsa_version(void);

@@ -2,6 +2,7 @@
 // TMA tensor-map encoding, workspace carving and stream-ordered launches of the
 // DSA kernels. Nothing here computes a step of the method; every step runs in
 // the kernels. No device memory is allocated on these paths.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -19,6 +20,7 @@ __device__ int g_dsa_status;
 namespace {
 
 thread_local int32_t t_last_cuda_error = 0;
+std::atomic<int64_t> g_launches{0};
 
 constexpr int kMaxDevices = 64;
 constexpr int kKMax = 2048;
@@ -41,6 +43,14 @@ dsa_status cuda_fail(cudaError_t e) {
   do {                                              \
     cudaError_t e_ = (expr);                        \
     if (e_ != cudaSuccess) return cuda_fail(e_);    \
+  } while (0)
+
+// A kernel launch through one of the dsa::launch_* helpers, counted.
+#define DSA_LAUNCH(expr)                            \
+  do {                                              \
+    cudaError_t e_ = (expr);                        \
+    if (e_ != cudaSuccess) return cuda_fail(e_);    \
+    g_launches.fetch_add(1, std::memory_order_relaxed); \
   } while (0)
 
 #define DSA_TRY(expr)                               \
@@ -269,7 +279,7 @@ dsa_status run_indexer(const dsa_indexer_in& in, const int32_t* rows, int32_t q_
     a.n_cols = n_cols;
     a.write_masked = write_masked;
     a.status = dev->status;
-    DSA_TRY_CUDA(dsa::launch_indexer_fp8(a, dev->num_sms, stream));
+    DSA_LAUNCH(dsa::launch_indexer_fp8(a, dev->num_sms, stream));
     return DSA_OK;
   }
   dsa::IndexerF32Args a{};
@@ -287,7 +297,7 @@ dsa_status run_indexer(const dsa_indexer_in& in, const int32_t* rows, int32_t q_
   a.ld_scores = ld_scores;
   a.n_cols = n_cols;
   a.status = dev->status;
-  DSA_TRY_CUDA(dsa::launch_indexer_f32(a, stream));
+  DSA_LAUNCH(dsa::launch_indexer_f32(a, stream));
   return DSA_OK;
 }
 
@@ -305,7 +315,7 @@ dsa_status run_topk(const float* scores, int64_t ld_scores, const int32_t* row_p
   a.idx = idx;
   a.ld_idx = ld_idx;
   a.status = dev->status;
-  DSA_TRY_CUDA(dsa::launch_topk(a, stream));
+  DSA_LAUNCH(dsa::launch_topk(a, stream));
   return DSA_OK;
 }
 
@@ -338,7 +348,7 @@ dsa_status run_attn(const dsa_attn_in& in, const int32_t* idx, int64_t ld_idx, i
     a.out = static_cast<__nv_bfloat16*>(out);
     a.lse = lse;
     a.status = dev->status;
-    DSA_TRY_CUDA(dsa::launch_attn_bf16(a, stream));
+    DSA_LAUNCH(dsa::launch_attn_bf16(a, stream));
     return DSA_OK;
   }
   dsa::AttnF32Args a{};
@@ -359,7 +369,29 @@ dsa_status run_attn(const dsa_attn_in& in, const int32_t* idx, int64_t ld_idx, i
   a.out = static_cast<float*>(out);
   a.lse = lse;
   a.status = dev->status;
-  DSA_TRY_CUDA(dsa::launch_attn_f32(a, stream));
+  DSA_LAUNCH(dsa::launch_attn_f32(a, stream));
+  return DSA_OK;
+}
+
+// Indexer -> top-k over bounded blocks of query rows (prefill) or all rows at
+// once (paged decode: one row per sequence), scores living only in `scores`.
+dsa_status run_select(const dsa_indexer_in& ind, int32_t k, int32_t* idx, int64_t ld_idx,
+                      float* scores, const ForwardPlan& p, DeviceInfo* dev,
+                      cudaStream_t stream) {
+  const int32_t n_q = ind.n_q;
+  if (ind.kv.kind == DSA_KV_PAGED) {
+    DSA_TRY(run_indexer(ind, nullptr, 0, n_q, scores, p.n_cols, p.n_cols, 0, dev, stream));
+    // query b sits at position ctx_lens[b] - 1
+    return run_topk(scores, p.n_cols, ind.kv.ctx_lens, 1, 0, n_q, k, idx, ld_idx, dev, stream);
+  }
+  const int32_t off = ind.n_keys - n_q;  // position of query 0
+  for (int32_t q0 = 0; q0 < n_q; q0 += p.chunk) {
+    const int32_t rows = n_q - q0 < p.chunk ? n_q - q0 : p.chunk;
+    const int32_t cols = off + q0 + rows;  // keys any query of the block sees
+    DSA_TRY(run_indexer(ind, nullptr, q0, rows, scores, cols, cols, 0, dev, stream));
+    DSA_TRY(run_topk(scores, cols, nullptr, 0, off + q0, rows, k,
+                     idx + static_cast<int64_t>(q0) * ld_idx, ld_idx, dev, stream));
+  }
   return DSA_OK;
 }
 
@@ -424,11 +456,12 @@ DSA_API dsa_status dsa_workspace_size(int32_t op, const dsa_indexer_in* indexer,
     case DSA_OP_TOPK:
     case DSA_OP_SPARSE_MQA:
       return DSA_OK;
-    case DSA_OP_FORWARD: {
+    case DSA_OP_FORWARD:
+    case DSA_OP_SELECT: {
       DSA_TRY(check_indexer(indexer));
       if (k < 1 || k > kKMax) return DSA_ERR_INVALID_ARG;
       const ForwardPlan p = forward_plan(*indexer, k);
-      *bytes = p.scores_bytes + p.idx_bytes;
+      *bytes = p.scores_bytes + (op == DSA_OP_FORWARD ? p.idx_bytes : 0);
       return DSA_OK;
     }
     default:
@@ -460,26 +493,26 @@ DSA_API dsa_status dsa_forward(const dsa_indexer_in* indexer, const dsa_attn_in*
   DeviceInfo* dev = nullptr;
   DSA_TRY(device_info(&dev));
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  float* scores = static_cast<float*>(ws);
   int32_t* idx = idx_out ? idx_out
                          : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + p.scores_bytes);
-  const int32_t n_q = indexer->n_q;
-  if (paged) {
-    DSA_TRY(run_indexer(*indexer, nullptr, 0, n_q, scores, p.n_cols, p.n_cols, 0, dev, stream));
-    // query b sits at position ctx_lens[b] - 1
-    DSA_TRY(run_topk(scores, p.n_cols, indexer->kv.ctx_lens, 1, 0, n_q, k, idx, k, dev, stream));
-  } else {
-    const int32_t off = indexer->n_keys - n_q;  // position of query 0
-    for (int32_t q0 = 0; q0 < n_q; q0 += p.chunk) {
-      const int32_t rows = n_q - q0 < p.chunk ? n_q - q0 : p.chunk;
-      const int32_t cols = off + q0 + rows;    // keys any query of the block sees
-      DSA_TRY(run_indexer(*indexer, nullptr, q0, rows, scores, cols, cols, 0, dev, stream));
-      DSA_TRY(run_topk(scores, cols, nullptr, 0, off + q0, rows, k,
-                       idx + static_cast<int64_t>(q0) * k, k, dev, stream));
-    }
-  }
+  DSA_TRY(run_select(*indexer, k, idx, k, static_cast<float*>(ws), p, dev, stream));
   return run_attn(*attn, idx, k, k, out, lse, dev, stream);
 }
+
+DSA_API dsa_status dsa_select(const dsa_indexer_in* indexer, int32_t k, int32_t* idx,
+                              int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  DSA_TRY(check_indexer(indexer));
+  if (idx == nullptr || k < 1 || k > kKMax || ld_idx < k) return DSA_ERR_INVALID_ARG;
+  const ForwardPlan p = forward_plan(*indexer, k);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < p.scores_bytes)
+    return DSA_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  DSA_TRY(device_info(&dev));
+  return run_select(*indexer, k, idx, ld_idx, static_cast<float*>(ws), p, dev,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+DSA_API int64_t dsa_launch_counter(void) { return g_launches.load(); }
 
 DSA_API dsa_status dsa_check_status(dsa_stream_t stream) {
   DeviceInfo* dev = nullptr;

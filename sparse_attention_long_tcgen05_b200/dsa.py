@@ -29,9 +29,11 @@ DSA_F32, DSA_E4M3, DSA_BF16 = 0, 1, 2
 DSA_KV_CONTIGUOUS, DSA_KV_PAGED = 0, 1
 DSA_OP_INDEXER_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MQA, DSA_OP_FORWARD = 0, 1, 2, 3
 
-EXPORTED = ["dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_fwd", "dsa_forward",
+DSA_OP_SELECT = 4
+
+EXPORTED = ["dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_fwd", "dsa_select", "dsa_forward",
             "dsa_workspace_size", "dsa_check_status", "dsa_status_string",
-            "dsa_last_cuda_error", "dsa_version"]
+            "dsa_last_cuda_error", "dsa_launch_counter", "dsa_version"]
 
 
 class DsaError(RuntimeError):
@@ -75,7 +77,9 @@ def _load():
         "dsa_indexer_scores": [ctypes.POINTER(IndexerIn), P, I32, P, I64, I32, P, SZ, P],
         "dsa_topk": [P, I64, P, I32, I32, P, I64, P],
         "dsa_sparse_mqa_fwd": [ctypes.POINTER(AttnIn), P, I64, I32, P, P, P, SZ, P],
+        "dsa_select": [ctypes.POINTER(IndexerIn), I32, P, I64, P, SZ, P],
         "dsa_forward": [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), I32, P, P, P, P, SZ, P],
+        "dsa_launch_counter": [],
         "dsa_workspace_size": [I32, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), I32, I32,
                                I32, ctypes.POINTER(SZ)],
         "dsa_check_status": [P],
@@ -86,7 +90,8 @@ def _load():
     for name, args in sig.items():
         f = getattr(lib, name)
         f.argtypes = args
-        f.restype = ctypes.c_char_p if name == "dsa_status_string" else ctypes.c_int32
+        f.restype = {"dsa_status_string": ctypes.c_char_p,
+                     "dsa_launch_counter": ctypes.c_int64}.get(name, ctypes.c_int32)
     return lib
 
 
@@ -193,6 +198,15 @@ def dsa_sparse_mqa_fwd(attn: _Keep, idx: torch.Tensor, k: int, out: torch.Tensor
                                   _ptr(out), _ptr(lse), _ptr(ws),
                                   0 if ws is None else ws.numel() * ws.element_size(),
                                   _stream(stream)), "dsa_sparse_mqa_fwd")
+
+
+def dsa_select(ind: _Keep, k: int, idx: torch.Tensor, ws: torch.Tensor, stream=None):
+    _check(LIB.dsa_select(ctypes.byref(ind.struct), k, _ptr(idx), idx.stride(0), _ptr(ws),
+                          ws.numel() * ws.element_size(), _stream(stream)), "dsa_select")
+
+
+def dsa_launch_counter() -> int:
+    return int(LIB.dsa_launch_counter())
 
 
 def dsa_forward(ind: _Keep, attn: _Keep, k: int, idx_out: Optional[torch.Tensor],

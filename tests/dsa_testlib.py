@@ -35,7 +35,7 @@ def assert_indexer_close(g, o, rel=IDX_REL, floor=IDX_FLOOR):
     assert np.all(np.isfinite(g[fin]))
     rowmax = np.max(np.where(fin, np.abs(o), 0.0), axis=1, keepdims=True)
     bound = rel * np.maximum(np.abs(o), floor * rowmax)
-    err = np.abs(g - o)
+    err = np.abs(np.where(fin, g, 0.0) - np.where(fin, o, 0.0))
     bad = fin & (err > bound)
     assert not bad.any(), (f"{bad.sum()} indexer entries out of tolerance; worst "
                            f"{np.max(np.where(fin, err / np.maximum(bound, 1e-30), 0)):.3g}x bound")
