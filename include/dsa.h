@@ -205,6 +205,34 @@ DSA_API const char* dsa_status_string(dsa_status status);
 /* The cudaError_t value behind the last DSA_ERR_CUDA on this thread (0 if none). */
 DSA_API int32_t dsa_last_cuda_error(void);
 
+/* Allocation-free form of dsa_select (the paper has no counterpart; this is a
+ * service for callers that cannot allocate device memory).
+ *
+ * Some callers cannot hand this library a workspace: a plugin that a host
+ * application (a serving engine, another language's runtime) loads and gives
+ * only its input and output buffers, because the host owns every byte of
+ * device memory through its own pool; or a latency-critical loop that must not
+ * call cudaMalloc, which can synchronise the whole device. This entry point
+ * takes no workspace and allocates nothing: its score rows live in a fixed
+ * 16 MiB scratch array that the library keeps in device memory (one per GPU
+ * that loads the library, held until the process exits).
+ *
+ * Same arguments and results as dsa_select (bit-identical idx), minus the
+ * workspace. Query rows are processed in blocks that fit the scratch, so one
+ * score row -- n_keys floats (CONTIGUOUS) or max_pages*page_size floats
+ * (PAGED) -- must fit in 16 MiB, i.e. at most 4,194,304 keys; larger problems
+ * return DSA_ERR_WORKSPACE_TOO_SMALL without launching anything.
+ *
+ * The first call on each device looks up the scratch array's device address
+ * (with that device current); make that first call before any stream capture.
+ * Every call on a device shares the one scratch array and leaves its last
+ * contents in it; no call relies on what an earlier call left there. Calls
+ * whose kernels overlap on the same device (other streams or threads) race on
+ * the scratch and give wrong results: order them. */
+#define DSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+DSA_API dsa_status dsa_select_noalloc(const dsa_indexer_in* indexer, int32_t k, int32_t* idx,
+                                      int64_t ld_idx, dsa_stream_t stream);
+
 /* Number of kernel launches this process has issued through the library so
  * far (all devices, all threads). Lets a caller count launches in a region. */
 DSA_API int64_t dsa_launch_counter(void);

@@ -545,3 +545,84 @@ DSA_API int32_t dsa_last_cuda_error(void) { return t_last_cuda_error; }
 DSA_API int32_t dsa_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free selection (dsa_select_noalloc). For callers that cannot hand
+// the library a workspace -- a plugin whose host owns all device memory through
+// its own pool, or a loop that must not call cudaMalloc because it can
+// synchronise the device -- the score rows of one block of queries live in this
+// fixed file-scope array instead. It is 16 MiB on every GPU that loads the
+// library, kept until the process exits. Host code must not pass its name to a
+// kernel (on the host it names a stand-in, not device memory): the device
+// address is looked up once per device below and passed explicitly.
+
+namespace {
+
+static __device__ __align__(256) float
+    g_noalloc_scratch[DSA_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+struct NoallocScratch {
+  bool init = false;
+  float* ptr = nullptr;
+};
+NoallocScratch g_noalloc[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device; the first call on
+// a device looks it up (with that device current) and caches it.
+dsa_status noalloc_scratch(float** out) {
+  int dev = 0;
+  DSA_TRY_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoallocScratch& s = g_noalloc[dev];
+  if (!s.init) {
+    void* p = nullptr;
+    DSA_TRY_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    s.ptr = static_cast<float*>(p);
+    s.init = true;
+  }
+  *out = s.ptr;
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" DSA_API dsa_status dsa_select_noalloc(const dsa_indexer_in* indexer, int32_t k,
+                                                 int32_t* idx, int64_t ld_idx,
+                                                 dsa_stream_t stream_) {
+  DSA_TRY(check_indexer(indexer));
+  if (idx == nullptr || k < 1 || k > kKMax || ld_idx < k) return DSA_ERR_INVALID_ARG;
+  const bool paged = indexer->kv.kind == DSA_KV_PAGED;
+  const int64_t n_cols = paged ? static_cast<int64_t>(indexer->kv.max_pages) * kPage
+                               : static_cast<int64_t>(indexer->n_keys);
+  const int64_t cap = DSA_NOALLOC_SCRATCH_BYTES / sizeof(float);
+  if (n_cols > cap) return DSA_ERR_WORKSPACE_TOO_SMALL;  // one score row must fit
+  DeviceInfo* dev = nullptr;
+  DSA_TRY(device_info(&dev));
+  float* scratch = nullptr;
+  DSA_TRY(noalloc_scratch(&scratch));
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const int32_t n_q = indexer->n_q;
+  int64_t block = cap / n_cols;            // query rows whose scores fit at once
+  if (block >= 4) block -= block % 4;
+  if (block > n_q) block = n_q;
+  // Every score the top-k reads (columns 0..pos of each row of the block) is
+  // written by the indexer launch just before it, so nothing needs clearing.
+  for (int32_t q0 = 0; q0 < n_q; q0 += static_cast<int32_t>(block)) {
+    const int32_t rows = static_cast<int32_t>(n_q - q0 < block ? n_q - q0 : block);
+    int32_t* out = idx + static_cast<int64_t>(q0) * ld_idx;
+    if (paged) {
+      const int32_t cols = static_cast<int32_t>(n_cols);
+      DSA_TRY(run_indexer(*indexer, nullptr, q0, rows, scratch, cols, cols, 0, dev, stream));
+      DSA_TRY(run_topk(scratch, cols, indexer->kv.ctx_lens + q0, 1, 0, rows, k, out, ld_idx, dev,
+                       stream));
+    } else {
+      const int32_t off = indexer->n_keys - n_q;
+      const int32_t cols = off + q0 + rows;
+      DSA_TRY(run_indexer(*indexer, nullptr, q0, rows, scratch, cols, cols, 0, dev, stream));
+      DSA_TRY(run_topk(scratch, cols, nullptr, 0, off + q0, rows, k, out, ld_idx, dev, stream));
+    }
+  }
+  return DSA_OK;
+}

@@ -33,7 +33,7 @@ DSA_OP_SELECT = 4
 
 EXPORTED = ["dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_fwd", "dsa_select", "dsa_forward",
             "dsa_workspace_size", "dsa_check_status", "dsa_status_string",
-            "dsa_last_cuda_error", "dsa_launch_counter", "dsa_version"]
+            "dsa_last_cuda_error", "dsa_launch_counter", "dsa_version", "dsa_select_noalloc"]
 
 
 class DsaError(RuntimeError):
@@ -80,6 +80,7 @@ def _load():
         "dsa_select": [ctypes.POINTER(IndexerIn), I32, P, I64, P, SZ, P],
         "dsa_forward": [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), I32, P, P, P, P, SZ, P],
         "dsa_launch_counter": [],
+        "dsa_select_noalloc": [ctypes.POINTER(IndexerIn), I32, P, I64, P],
         "dsa_workspace_size": [I32, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), I32, I32,
                                I32, ctypes.POINTER(SZ)],
         "dsa_check_status": [P],
@@ -203,6 +204,14 @@ def dsa_sparse_mqa_fwd(attn: _Keep, idx: torch.Tensor, k: int, out: torch.Tensor
 def dsa_select(ind: _Keep, k: int, idx: torch.Tensor, ws: torch.Tensor, stream=None):
     _check(LIB.dsa_select(ctypes.byref(ind.struct), k, _ptr(idx), idx.stride(0), _ptr(ws),
                           ws.numel() * ws.element_size(), _stream(stream)), "dsa_select")
+
+
+def dsa_select_noalloc(ind: _Keep, k: int, idx: torch.Tensor, stream=None):
+    """dsa_select without a workspace, for callers that cannot allocate device
+    memory: the library's fixed 16 MiB per-GPU scratch holds the score rows.
+    Calls on one device must not overlap (they share that scratch)."""
+    _check(LIB.dsa_select_noalloc(ctypes.byref(ind.struct), k, _ptr(idx), idx.stride(0),
+                                  _stream(stream)), "dsa_select_noalloc")
 
 
 def dsa_launch_counter() -> int:
