@@ -215,6 +215,9 @@ def run_ours(args, world, rank, local):
 
     peaks = load_peaks()
     fp8_sustained = 2.0 * peaks["bf16_sustained"]   # FP8 dense = 2x bf16 (nominal ratio)
+    if args.decode_only:    # profiling aid: the decode step alone
+        return {"decode": run_decode(args, world, rank, local, peaks, dsa, make_decode,
+                                     WORKLOADS[DECODE_WL])}
     wl = next(w for w in WORKLOADS.values() if w.name == args.workload)
     L, k = wl.L, wl.k
     inp = make_prefill(wl, device="cuda", seed=rank)
@@ -472,6 +475,8 @@ def main():
                     choices=["prefill_L4096", "prefill_L32768_needle", "prefill_L131072"],
                     help="prefill workload of the headline line (smaller ones for profiling)")
     ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode step (profiling aid; no headline value)")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)

@@ -170,7 +170,8 @@ dsa_status check_indexer(const dsa_indexer_in* in) {
   if (in->dtype == DSA_E4M3) {
     if (!is_fp8_indexer(*in)) return DSA_ERR_UNSUPPORTED;
     if (in->q_scale == nullptr || in->k_scale == nullptr) return DSA_ERR_INVALID_ARG;
-    if (!aligned16(in->q) || !aligned16(in->k) || in->ld_q % 16 || in->ld_k % 16)
+    if (!aligned16(in->q) || !aligned16(in->k) || !aligned16(in->k_scale) || in->ld_q % 16 ||
+        in->ld_k % 16)
       return DSA_ERR_INVALID_ARG;
     return DSA_OK;
   }
@@ -267,6 +268,10 @@ dsa_status run_indexer(const dsa_indexer_in& in, const int32_t* rows, int32_t q_
       const uint32_t box[2] = {128, ks.paged ? 64u : 128u};
       DSA_TRY(make_map(&a.map_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, in.k, dims, strides, box,
                        CU_TENSOR_MAP_SWIZZLE_128B));
+      const uint64_t sdims[1] = {rows_k};
+      const uint32_t sbox[1] = {ks.paged ? 64u : 128u};
+      DSA_TRY(make_map(&a.map_sk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, in.k_scale, sdims, nullptr,
+                       sbox, CU_TENSOR_MAP_SWIZZLE_NONE));
     }
     a.q_scale = in.q_scale;
     a.w = in.w;
@@ -324,13 +329,8 @@ dsa_status run_attn(const dsa_attn_in& in, const int32_t* idx, int64_t ld_idx, i
   const dsa::KeySide ks = key_side(in.kv_layout, in.n_q, in.n_keys);
   if (in.dtype == DSA_BF16) {
     dsa::AttnBf16Args a{};
-    {
-      const uint64_t dims[3] = {576, 128, static_cast<uint64_t>(in.n_q)};
-      const uint64_t strides[2] = {576 * 2, static_cast<uint64_t>(in.ld_q) * 2};
-      const uint32_t box[3] = {64, 128, 1};
-      DSA_TRY(make_map(&a.map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, in.q, dims, strides, box,
-                       CU_TENSOR_MAP_SWIZZLE_128B));
-    }
+    a.q = static_cast<const __nv_bfloat16*>(in.q);
+    a.ld_q = in.ld_q;
     {
       const uint64_t rows_kv = ks.paged ? static_cast<uint64_t>(in.kv_layout.num_pages) * kPage
                                         : static_cast<uint64_t>(in.n_keys);

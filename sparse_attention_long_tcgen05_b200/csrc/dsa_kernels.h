@@ -34,6 +34,7 @@ struct KeySide {
 struct IndexerFp8Args {
   CUtensorMap map_q;   // 3-D {d=128, heads=64, n_q} e4m3, box {128,64,1}, 128B swizzle
   CUtensorMap map_k;   // 2-D {128, key rows}, box {128, 128} (contiguous) or {128, 64} (paged)
+  CUtensorMap map_sk;  // 1-D {key rows} f32 key scales, box {128} (contiguous) or {64} (paged)
   const float* q_scale;
   const float* w;
   int64_t ld_w;
@@ -87,8 +88,9 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
 // ---------------------------------------------------------------- attention
 
 struct AttnBf16Args {
-  CUtensorMap map_q;    // 3-D {576, 128, n_q} bf16, box {64, 128, 1}, 128B swizzle
-  CUtensorMap map_kv;   // 2-D {576, kv rows} bf16, box {64, 1}, 128B swizzle (gather4)
+  CUtensorMap map_kv;      // 2-D {576, kv rows} bf16, box {64, 1}, 128B swizzle (gather4)
+  const __nv_bfloat16* q;  // [n_q, 128, 576], 16-byte aligned rows
+  int64_t ld_q;            // elements between query tokens
   const int32_t* idx;
   int64_t ld_idx;
   int32_t k;

@@ -10,16 +10,20 @@
 // per-token scales (q = sq[t] * code, k = sk[s] * code) this is
 //     I[t,s] = sk[s] * sum_j (w[t,j] * sq[t]) * ReLU(code_q[t,j] . code_k[s]),
 // which is what the kernel evaluates: the code dot products on the tensor core
-// (exact e4m3 products, f32 accumulation), then the epilogue below.
+// (exact e4m3 products, f32 accumulation), then the epilogue of
+// indexer_epilogue.cuh.
 //
 // Mapping: one MMA is D[128 keys, G*64] = K_tile[128 x 128 B] * Qgroup[G*64 x 128 B]^T
 // with keys on TMEM lanes and (query, head) on TMEM columns, so each epilogue
 // thread owns one key and reduces the 64 heads of a query inside its registers.
 //
-// Roles (192 threads, one CTA per SM, persistent over work units):
-//   warp 0    TMA producer: Q group (once per unit) and key tiles (6-stage ring)
+// Roles (320 threads, one CTA per SM, persistent over work units):
+//   warp 0    TMA producer: Q group (once per unit), key tiles and their fp32
+//             key scales through a 6-stage ring
 //   warp 1    TMEM owner and single-thread MMA issuer (2 accumulators in TMEM)
-//   warps 2-5 epilogue: tcgen05.ld -> ReLU * w -> head sum -> * sk -> global
+//   warps 2-9 epilogue, two warps per TMEM sub-partition: warps 2-5 reduce
+//             queries 0-1 of the group, warps 6-9 queries 2-3;
+//             tcgen05.ld -> ReLU * w -> head sum -> * sk -> global
 // A work unit is (group of G query rows, run of up to 16 key tiles of 128).
 #include "dsa_common.cuh"
 #include "dsa_kernels.h"
@@ -34,14 +38,18 @@ constexpr int kKeyTile = 128;
 constexpr int kMaxG = 4;
 constexpr int kStages = 6;
 constexpr int kTilesPerUnit = 16;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kThreads = 64 + kEpiThreads;
 constexpr int kQBytes = kHeads * kDim;      // 8 KB per query
 constexpr int kKBytes = kKeyTile * kDim;    // 16 KB per key tile
+constexpr int kSkBytes = kKeyTile * 4;      // 512 B of key scales per tile
 constexpr uint32_t kTmemCols = 512;
 
 struct __align__(1024) Smem {
   uint8_t q[2][kMaxG * kQBytes];     // B operand (query group), double buffered per unit
   uint8_t k[kStages][kKBytes];       // A operand (key tile) ring
+  float sk[kStages][kKeyTile];       // key scales of the tile in the same stage
   float wq[kMaxG * kHeads];          // w[t,j] * sq[t] of the current unit
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[kStages], k_empty[kStages];
@@ -125,17 +133,20 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
       mbar_init(&S.q_full[i], 1);
       mbar_init(&S.q_empty[i], 1);
       mbar_init(&S.acc_full[i], 1);
-      mbar_init(&S.acc_empty[i], 128);
+      mbar_init(&S.acc_empty[i], kEpiThreads);
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&S.k_full[i], 1);
-      mbar_init(&S.k_empty[i], 1);
+      // released by the MMAs' completion and by every epilogue thread once it
+      // has read the stage's key scales
+      mbar_init(&S.k_empty[i], 1 + kEpiThreads);
     }
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&a.map_q);
     tma_prefetch_desc(&a.map_k);
+    tma_prefetch_desc(&a.map_sk);
   }
   if (warp == 1) tmem_alloc(&S.tmem_base, kTmemCols);
   tc_fence_before();
@@ -159,15 +170,18 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           tma_load_3d(S.q[qb] + i * kQBytes, &a.map_q, 0, 0, U.qi[i], &S.q_full[qb]);
         for (int t = U.t0; t < U.t_end; ++t) {
           if (!mbar_wait(&S.k_empty[ks], kph ^ 1, a.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&S.k_full[ks], kKBytes);
+          mbar_arrive_expect_tx(&S.k_full[ks], kKBytes + kSkBytes);
           if (!a.keys.paged) {
             tma_load_2d(S.k[ks], &a.map_k, 0, t * kKeyTile, &S.k_full[ks]);
+            tma_load_1d(S.sk[ks], &a.map_sk, t * kKeyTile, &S.k_full[ks]);
           } else {
             const int p0 = 2 * t;
             const int pg0 = page_of(a, U.qi[0], p0, true);
             const int pg1 = (p0 + 1) * 64 <= U.max_pos ? page_of(a, U.qi[0], p0 + 1, true) : pg0;
             tma_load_2d(S.k[ks], &a.map_k, 0, pg0 * 64, &S.k_full[ks]);
             tma_load_2d(S.k[ks] + kKBytes / 2, &a.map_k, 0, pg1 * 64, &S.k_full[ks]);
+            tma_load_1d(S.sk[ks], &a.map_sk, pg0 * 64, &S.k_full[ks]);
+            tma_load_1d(S.sk[ks] + 64, &a.map_sk, pg1 * 64, &S.k_full[ks]);
           }
           if (++ks == kStages) { ks = 0; kph ^= 1; }
         }
@@ -207,55 +221,73 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
   } else {
     // ------------------------------------------------------------ epilogue
     const int sub = warp & 3;              // TMEM sub-partition of this warp
-    const int et = threadIdx.x - 64;       // 0..127
-    int ab = 0;
-    uint32_t aph = 0;
+    const int half = (warp - 2) >> 2;      // 0: queries 0-1, 1: queries 2-3
+    const int et = threadIdx.x - 64;       // 0..255
+    int ab = 0, ks = 0;
+    uint32_t aph = 0, kph = 0;
     // After a timed-out wait the warp stops waiting and computing but keeps
     // walking the same units, so every epilogue warp meets every named barrier.
     bool ok = true;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       const Unit U = get_unit(a, G, n_chunks, n_tiles, u, false);
-      named_bar_sync(1, 128);
-      for (int i = et; i < U.ng * kHeads; i += 128) {
+      named_bar_sync(1, kEpiThreads);
+      for (int i = et; i < U.ng * kHeads; i += kEpiThreads) {
         const int g = i / kHeads;
         const int qi = U.qi[g];
         S.wq[i] = a.w[static_cast<int64_t>(qi) * a.ld_w + (i % kHeads)] * a.q_scale[qi];
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, kEpiThreads);
+      const int g0 = 2 * half;                          // first query of this warp
+      const int nq = max(0, min(2, U.ng - g0));         // queries this warp reduces
       for (int t = U.t0; t < U.t1 && ok; ++t) {
         const int s = t * kKeyTile + sub * 32 + lane;
         if (t >= U.t_end) {
           if (a.write_masked && s < a.n_cols)
-            for (int g = 0; g < U.ng; ++g)
-              a.scores[static_cast<int64_t>(U.row0 + g) * a.ld_scores + s] = -INFINITY;
+            for (int gq = 0; gq < nq; ++gq)
+              a.scores[static_cast<int64_t>(U.row0 + g0 + gq) * a.ld_scores + s] = -INFINITY;
           continue;
         }
-        // key scale (0 for keys no query of the group sees)
-        float sk = 0.f;
-        if (s <= U.max_pos) {
-          if (!a.keys.paged) {
-            sk = a.k_scale[s];
-          } else {
-            const int pg = page_of(a, U.qi[0], s >> 6, false);
-            sk = a.k_scale[static_cast<int64_t>(pg) * 64 + (s & 63)];
-          }
-        }
+        // this tile's key scale (the stage also holds the key codes)
+        if (!mbar_wait_warp(&S.k_full[ks], kph, a.status)) { ok = false; break; }
+        const float sk = S.sk[ks][sub * 32 + lane];
+        mbar_arrive(&S.k_empty[ks]);
+        if (++ks == kStages) { ks = 0; kph ^= 1; }
         if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t tbase =
-            tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(ab * N);
-        for (int g = 0; g < U.ng; ++g) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tbase + g * kHeads, r0);
-          tmem_ld32(tbase + g * kHeads + 32, r1);
+        const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) +
+                               static_cast<uint32_t>(ab * N + g0 * kHeads);
+        if (nq == 2) {
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(tbase, r0);
+          tmem_ld32(tbase + 32, r1);
+          tmem_ld32(tbase + 64, r2);
+          tmem_ld32(tbase + 96, r3);
           tmem_wait_ld();
-          const float score = indexer_score_from_dots(r0, r1, &S.wq[g * kHeads], sk);
+          tc_fence_before();
+          mbar_arrive(&S.acc_empty[ab]);
+          const float s0 = indexer_score_from_dots(r0, r1, &S.wq[g0 * kHeads], sk);
+          const float s1 = indexer_score_from_dots(r2, r3, &S.wq[(g0 + 1) * kHeads], sk);
+          if (s < a.n_cols) {
+            a.scores[static_cast<int64_t>(U.row0 + g0) * a.ld_scores + s] =
+                s <= U.pos[g0] ? s0 : -INFINITY;
+            a.scores[static_cast<int64_t>(U.row0 + g0 + 1) * a.ld_scores + s] =
+                s <= U.pos[g0 + 1] ? s1 : -INFINITY;
+          }
+        } else if (nq == 1) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tbase, r0);
+          tmem_ld32(tbase + 32, r1);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&S.acc_empty[ab]);
+          const float s0 = indexer_score_from_dots(r0, r1, &S.wq[g0 * kHeads], sk);
           if (s < a.n_cols)
-            a.scores[static_cast<int64_t>(U.row0 + g) * a.ld_scores + s] =
-                s <= U.pos[g] ? score : -INFINITY;
+            a.scores[static_cast<int64_t>(U.row0 + g0) * a.ld_scores + s] =
+                s <= U.pos[g0] ? s0 : -INFINITY;
+        } else {
+          tc_fence_before();
+          mbar_arrive(&S.acc_empty[ab]);
         }
-        tc_fence_before();
-        mbar_arrive(&S.acc_empty[ab]);
         if (++ab == 2) { ab = 0; aph ^= 1; }
       }
     }

@@ -7,10 +7,18 @@
 // +0.0, NaN ranks below every number; the kept s are written in ascending
 // order, padded with -1 when t+1 < k.
 //
-// One CTA (1024 threads) per row: a three-digit MSB radix select (11/11/10
-// bits) over order-preserving uint32 keys finds the k-th largest key T and how
-// many keys equal to T are kept; a final stable compaction in index order
-// emits key > T, plus the first (lowest-index) keys == T.
+// One CTA (1024 threads) per row, scores compared as order-preserving uint32
+// keys. Two passes over the row:
+//   1. a histogram of the top 12 key bits finds the bin b1 holding the k-th
+//      largest key;
+//   2. an ordered collection (warp ballots, one block scan per 8192 scores)
+//      copies every key in a bin >= b1 -- the sure winners and the contenders
+//      of bin b1 -- with its index into shared memory, in index order.
+// The rest runs in shared memory: two 10-bit digits of the contenders give the
+// exact k-th key T and how many keys equal to T are kept; a stable compaction
+// of the collected list emits key > T plus the lowest-index keys == T.
+// If the collection would not fit (heavy ties), the row falls back to a
+// three-digit select with a compaction over the row in global memory.
 #include "dsa_common.cuh"
 #include "dsa_kernels.h"
 
@@ -19,6 +27,17 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
+constexpr int kPer = 8;                     // scores per lane per chunk
+constexpr int kChunk = kThreads * kPer;     // scores per block-scan
+constexpr int kCap = 14336;                 // collected (index, key) pairs
+
+struct TopkSmem {
+  uint32_t hist[4096];
+  uint32_t warp_sums[kWarps + 1];
+  uint32_t found[2];
+  int32_t lidx[kCap];
+  uint32_t lkey[kCap];
+};
 
 // Monotone map float -> uint32: a < b  <=>  key(a) < key(b); -0.0 -> key(+0.0);
 // NaN -> 0 (below -inf, whose key is 0x007fffff).
@@ -29,7 +48,7 @@ __device__ __forceinline__ uint32_t order_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Block-wide exclusive prefix sum; also returns the block total.
+// Block-wide exclusive prefix sum of one value per thread; also the total.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_sums,
                                                     uint32_t& total) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -42,7 +61,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_s
   if (lane == 31) warp_sums[w] = x;
   __syncthreads();
   if (w == 0) {
-    uint32_t s = warp_sums[lane];
+    const uint32_t s = warp_sums[lane];
     uint32_t t = s;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -59,12 +78,37 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_s
   return r;
 }
 
-// Given a histogram over `nb` bins of the candidates still in play and the
-// rank `k_rem` (1-based, from the top) being looked for, find the bin holding
-// it. Writes the bin and the rank inside that bin to out[0], out[1].
+// Exclusive prefix over the 32 warps of one value per warp (lane 0's `v`);
+// returns it to every lane of the warp, and the block total.
+__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t* warp_sums,
+                                                   uint32_t& total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (lane == 0) warp_sums[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    const uint32_t s = warp_sums[lane];
+    uint32_t t = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    warp_sums[lane] = t - s;
+    if (lane == 31) warp_sums[32] = t;
+  }
+  __syncthreads();
+  const uint32_t r = warp_sums[w];
+  total = warp_sums[32];
+  __syncthreads();
+  return r;
+}
+
+// Given a histogram over `nb` bins and the rank `k_rem` (1-based, from the
+// top) being looked for, find the bin holding it: out[0] = bin, out[1] = rank
+// inside that bin.
 __device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t k_rem,
                                          uint32_t* warp_sums, uint32_t* out) {
-  const int per = nb / kThreads;  // 1 or 2
+  const int per = nb / kThreads;  // 1, 2 or 4
   const int hi = nb - 1 - threadIdx.x * per;
   uint32_t local = 0;
   for (int i = 0; i < per; ++i) local += hist[hi - i];
@@ -81,17 +125,101 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t 
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
-  __shared__ uint32_t hist[2048];
-  __shared__ uint32_t warp_sums[kWarps + 1];
-  __shared__ uint32_t found[2];
+__device__ __forceinline__ void clear_hist(uint32_t* hist, int nb) {
+  for (int i = threadIdx.x; i < nb; i += kThreads) hist[i] = 0;
+  __syncthreads();
+}
 
+// Ordered selection over `m` (index, key) pairs produced by `get(e)`, given the
+// threshold key T and the number of keys == T to keep: writes the kept indices
+// in the pairs' order to out[0..]. Pairs are taken kPer per lane, lane-major
+// inside a warp's 256-pair segment, so one block scan covers kChunk pairs.
+template <class Get>
+__device__ __forceinline__ void ordered_emit(int m, uint32_t T, uint32_t take_eq, int k,
+                                             int32_t* out, uint32_t* warp_sums, Get get) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t run_gt = 0, run_eq = 0;
+  for (int c0 = 0; c0 < m; c0 += kChunk) {
+    uint32_t bgt[kPer], beq[kPer];
+    int id[kPer];
+    uint32_t cgt = 0, ceq = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int e = c0 + w * (32 * kPer) + j * 32 + lane;
+      uint32_t key = 0;
+      id[j] = -1;
+      if (e < m) get(e, id[j], key);
+      const bool in = e < m;
+      bgt[j] = __ballot_sync(0xffffffffu, in && key > T);
+      beq[j] = __ballot_sync(0xffffffffu, in && key == T);
+      cgt += __popc(bgt[j]);
+      ceq += __popc(beq[j]);
+    }
+    uint32_t total;
+    const uint32_t ex = warp_excl_scan(cgt | (ceq << 16), warp_sums, total);
+    uint32_t gt_b = run_gt + (ex & 0xffffu);
+    uint32_t eq_b = run_eq + (ex >> 16);
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const uint32_t g_me = gt_b + __popc(bgt[j] & lt);
+      const uint32_t e_me = eq_b + __popc(beq[j] & lt);
+      const bool gt = (bgt[j] >> lane) & 1u;
+      const bool eq = (beq[j] >> lane) & 1u;
+      if (gt || (eq && e_me < take_eq)) out[g_me + min(e_me, take_eq)] = id[j];
+      gt_b += __popc(bgt[j]);
+      eq_b += __popc(beq[j]);
+    }
+    run_gt += total & 0xffffu;
+    run_eq += total >> 16;
+    if (run_gt + min(run_eq, take_eq) >= static_cast<uint32_t>(k)) break;
+  }
+}
+
+// Exact select without the shared-memory collection (rows with heavy ties):
+// digits 11/11/10 over the row in global memory, then an ordered compaction of
+// the row.
+__device__ void select_in_global(const float* row, int n, int k, int32_t* out, TopkSmem& S) {
+  clear_hist(S.hist, 2048);
+  for (int i = threadIdx.x; i < n; i += kThreads) atomicAdd(&S.hist[order_key(row[i]) >> 21], 1u);
+  __syncthreads();
+  find_bin(S.hist, 2048, static_cast<uint32_t>(k), S.warp_sums, S.found);
+  uint32_t prefix = S.found[0];
+  uint32_t k_rem = S.found[1];
+  clear_hist(S.hist, 2048);
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    const uint32_t key = order_key(row[i]);
+    if ((key >> 21) == prefix) atomicAdd(&S.hist[(key >> 10) & 2047u], 1u);
+  }
+  __syncthreads();
+  find_bin(S.hist, 2048, k_rem, S.warp_sums, S.found);
+  prefix = (prefix << 11) | S.found[0];
+  k_rem = S.found[1];
+  clear_hist(S.hist, 1024);
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    const uint32_t key = order_key(row[i]);
+    if ((key >> 10) == prefix) atomicAdd(&S.hist[key & 1023u], 1u);
+  }
+  __syncthreads();
+  find_bin(S.hist, 1024, k_rem, S.warp_sums, S.found);
+  const uint32_t T = (prefix << 10) | S.found[0];
+  const uint32_t take_eq = S.found[1];
+  ordered_emit(n, T, take_eq, k, out, S.warp_sums, [&](int e, int& id, uint32_t& key) {
+    id = e;
+    key = order_key(row[e]);
+  });
+}
+
+__global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
   const int r = blockIdx.x;
   const int tid = threadIdx.x;
+  const int lane = tid & 31, w = tid >> 5;
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld_scores;
   int32_t* out = a.idx + static_cast<int64_t>(r) * a.ld_idx;
   const int pos = a.row_pos ? a.row_pos[r] - a.pos_minus : a.pos_base + r;
-  if (pos < 0) {
+  if (pos < 0 || pos >= a.ld_scores) {
     if (tid == 0) report(a.status, DSA_ERR_DEVICE_BOUNDS);
     for (int j = tid; j < a.k; j += kThreads) out[j] = -1;
     return;
@@ -103,66 +231,84 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
     return;
   }
 
-  // ---- digit 1: bits 31..21
-  for (int i = tid; i < 2048; i += kThreads) hist[i] = 0;
+  // ---- pass 1: histogram of the top 12 key bits
+  clear_hist(S.hist, 4096);
+  for (int i = tid; i < n; i += kThreads) atomicAdd(&S.hist[order_key(row[i]) >> 20], 1u);
   __syncthreads();
-  for (int i = tid; i < n; i += kThreads) atomicAdd(&hist[order_key(row[i]) >> 21], 1u);
-  __syncthreads();
-  find_bin(hist, 2048, static_cast<uint32_t>(k), warp_sums, found);
-  uint32_t prefix = found[0];
-  uint32_t k_rem = found[1];
-
-  // ---- digit 2: bits 20..10
-  for (int i = tid; i < 2048; i += kThreads) hist[i] = 0;
-  __syncthreads();
-  for (int i = tid; i < n; i += kThreads) {
-    const uint32_t key = order_key(row[i]);
-    if ((key >> 21) == prefix) atomicAdd(&hist[(key >> 10) & 2047u], 1u);
+  find_bin(S.hist, 4096, static_cast<uint32_t>(k), S.warp_sums, S.found);
+  const uint32_t b1 = S.found[0];
+  const uint32_t k_rem = S.found[1];
+  const uint32_t collect = static_cast<uint32_t>(k) - k_rem + S.hist[b1];
+  if (collect > static_cast<uint32_t>(kCap)) {   // uniform: every thread read the same values
+    select_in_global(row, n, k, out, S);
+    return;
   }
-  __syncthreads();
-  find_bin(hist, 2048, k_rem, warp_sums, found);
-  prefix = (prefix << 11) | found[0];
-  k_rem = found[1];
 
-  // ---- digit 3: bits 9..0
-  for (int i = tid; i < 1024; i += kThreads) hist[i] = 0;
-  __syncthreads();
-  for (int i = tid; i < n; i += kThreads) {
-    const uint32_t key = order_key(row[i]);
-    if ((key >> 10) == prefix) atomicAdd(&hist[key & 1023u], 1u);
-  }
-  __syncthreads();
-  find_bin(hist, 1024, k_rem, warp_sums, found);
-  const uint32_t T = (prefix << 10) | found[0];
-  const uint32_t take_eq = found[1];   // keys == T kept, lowest indices first
-
-  // ---- stable compaction in index order
-  uint32_t run_gt = 0, run_eq = 0;
-  for (int base = 0; base < n; base += kThreads) {
-    const int i = base + tid;
-    uint32_t gt = 0, eq = 0;
-    if (i < n) {
-      const uint32_t key = order_key(row[i]);
-      gt = key > T;
-      eq = key == T;
+  // ---- pass 2: collect keys in bins >= b1 with their indices, in index order
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t base = 0;
+  for (int c0 = 0; c0 < n; c0 += kChunk) {
+    uint32_t bal[kPer], key[kPer];
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = c0 + w * (32 * kPer) + j * 32 + lane;
+      key[j] = i < n ? order_key(row[i]) : 0u;
+      bal[j] = __ballot_sync(0xffffffffu, i < n && (key[j] >> 20) >= b1);
+      cnt += __popc(bal[j]);
     }
     uint32_t total;
-    const uint32_t ex = block_excl_scan(gt | (eq << 16), warp_sums, total);
-    const uint32_t gt_before = run_gt + (ex & 0xffffu);
-    const uint32_t eq_before = run_eq + (ex >> 16);
-    if (gt || (eq && eq_before < take_eq))
-      out[gt_before + min(eq_before, take_eq)] = i;
-    run_gt += total & 0xffffu;
-    run_eq += total >> 16;
-    if (run_gt + min(run_eq, take_eq) >= static_cast<uint32_t>(k)) break;
+    uint32_t off = base + warp_excl_scan(cnt, S.warp_sums, total);
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if ((bal[j] >> lane) & 1u) {
+        const uint32_t p = off + __popc(bal[j] & lt);
+        S.lidx[p] = c0 + w * (32 * kPer) + j * 32 + lane;
+        S.lkey[p] = key[j];
+      }
+      off += __popc(bal[j]);
+    }
+    base += total;
   }
+  __syncthreads();
+  const int m = static_cast<int>(base);
+
+  // ---- exact threshold among the contenders of bin b1 (shared memory only)
+  clear_hist(S.hist, 1024);
+  for (int e = tid; e < m; e += kThreads) {
+    const uint32_t kk = S.lkey[e];
+    if ((kk >> 20) == b1) atomicAdd(&S.hist[(kk >> 10) & 1023u], 1u);
+  }
+  __syncthreads();
+  find_bin(S.hist, 1024, k_rem, S.warp_sums, S.found);
+  const uint32_t p2 = (b1 << 10) | S.found[0];
+  const uint32_t k_rem2 = S.found[1];
+  clear_hist(S.hist, 1024);
+  for (int e = tid; e < m; e += kThreads) {
+    const uint32_t kk = S.lkey[e];
+    if ((kk >> 10) == p2) atomicAdd(&S.hist[kk & 1023u], 1u);
+  }
+  __syncthreads();
+  find_bin(S.hist, 1024, k_rem2, S.warp_sums, S.found);
+  const uint32_t T = (p2 << 10) | S.found[0];
+  const uint32_t take_eq = S.found[1];
+
+  // ---- ordered emit from the collected list
+  ordered_emit(m, T, take_eq, k, out, S.warp_sums, [&](int e, int& id, uint32_t& kk) {
+    id = S.lidx[e];
+    kk = S.lkey[e];
+  });
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   if (a.n_rows <= 0) return cudaSuccess;
-  topk_kernel<<<a.n_rows, kThreads, 0, stream>>>(a);
+  const size_t smem = sizeof(TopkSmem);
+  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  topk_kernel<<<a.n_rows, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 

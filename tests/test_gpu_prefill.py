@@ -118,6 +118,25 @@ def test_topk_ties_and_signed_zero(libs):
         assert np.array_equal(idx.cpu().numpy(), ref), k
 
 
+def test_topk_heavy_ties_fallback(libs):
+    """More tied contenders than the shared-memory collection holds: the exact
+    select over the row in global memory takes over and gives the same rule."""
+    dsa, T = libs
+    rng = np.random.default_rng(2)
+    R, n = 6, 30000
+    s = rng.choice(np.array([1.0, 2.0], dtype=np.float32), size=(R, n), p=[0.4, 0.6])
+    s[1] = 5.0
+    s[2, ::3] = 7.0
+    s[3] = rng.standard_normal(n).astype(np.float32)   # no ties: collection path
+    pos = np.array([n - 1, n - 1, 25000, n - 1, 15000, 2048], dtype=np.int32)
+    for k in (2048, 100):
+        idx = torch.empty(R, k, dtype=torch.int32, device="cuda")
+        dsa.dsa_topk(torch.from_numpy(s).cuda(), torch.from_numpy(pos).cuda(), k, idx)
+        assert dsa.dsa_check_status() == 0
+        ref = T.topk_oracle_on(s.astype(np.float64), pos, k)
+        assert np.array_equal(idx.cpu().numpy(), ref), k
+
+
 def _attention_case(dsa, T, L, k, seed, rows=None):
     inp = make_prefill(_wl(L, k), device="cuda", seed=seed)
     rng = np.random.default_rng(seed)
