@@ -13,35 +13,44 @@
 // TMEM columns of one SM, so one query runs on a CLUSTER OF TWO CTAs that split
 // the 576 key dimensions: CTA0 owns dims [0,256), CTA1 owns [256,576). Each CTA
 //   - keeps its slice of Q in TMEM (the MMA's A operand read from tensor
-//     memory), which leaves shared memory to a 4-deep ring of key blocks;
-//   - gathers only its column range of the selected rows with TMA tile::gather4
-//     (four 128-byte row pieces per request, 128B-swizzled on arrival, no
-//     multicast), so the pair reads each selected row exactly once. A request
-//     keeps its issuing warp busy ~90 cycles and the measured gather rate grows
-//     with the number of issuing warps, so 19 warps share the requests;
-//   - computes a partial S_r = Q[:, dims_r] K[:, dims_r]^T (M=128 heads,
-//     N=64 keys) into TMEM;
-//   - sends S_r to the peer (st.async into the peer's shared memory, counted on
-//     the peer's transaction barrier) and adds the peer's partial:
-//     S = S_0 + S_1 is bit-identical in both CTAs (fp32 addition commutes), so
-//     both run the same online softmax;
-//   - accumulates its half of the value columns, O[:, 256r : 256r+256] += P V_r,
-//     where V_r lies inside its own gathered columns (dims [256r, 256r+256)).
+//     memory) and gathers only its column range of the selected rows with TMA
+//     tile::gather4 (four 128-byte row pieces per request, 128B-swizzled on
+//     arrival, no multicast), so the pair reads each selected row once;
+//   - computes a partial S_r = Q[:, dims_r] K[:, dims_r]^T for all 128 heads
+//     (M=128, N=64 keys) into TMEM;
+//   - owns the softmax of 64 of the heads. TMEM lane 32s+i (i < 16) of SM
+//     sub-partition s holds one of its own heads, lane 32s+16+i one of the
+//     peer's; Q rows are staged in that order, so S, P and O rows follow it.
+//     The CTA sends the peer the 16 KB partial S of the peer's heads, adds
+//     the peer's partial for its own heads, runs the online softmax and
+//     writes the bf16 P rows of its heads into its own P tile, from where
+//     they are copied into the peer's (8 KB), together with the per-head
+//     rescale factors. Every transfer is a bulk copy out of this CTA's shared
+//     memory into the peer's, counted on the peer's transaction barrier: a
+//     few asynchronous operations per block, which leaves the SM's
+//     asynchronous copy path to the gather;
+//   - accumulates its half of the value columns, O[:, 256r : 256r+256] += P V_r
+//     for all 128 heads, where V_r lies inside its own gathered columns.
+// Measured on B200, cluster shared-memory traffic runs at ~20 B/cycle per SM
+// and direction, so the exchange is kept to the 24 KB per 64-key block that
+// the split requires, and QK^T of block j+1 is issued as soon as S_j has been
+// read, so that the partial S of block j+1 travels while block j's softmax runs.
 // The softmax keeps a stale running max and rescales O in TMEM only when the
 // block max exceeds it by more than 2^8 (exact: the final normalisation uses
-// the same max).
+// the same max); the owner of a head sends its factor to the peer, whose O
+// rows for that head are rescaled there.
 //
-// Roles per CTA (896 threads, 7 warps per SM sub-partition):
+// Roles per CTA (1024 threads, 8 warps per SM sub-partition):
 //   warps 0-15   plan (each scans two 64-entry blocks of the query's index row:
 //                physical rows, valid masks);
 //   warps 0-15, 17-19  issue the gather requests (lane 0 of each);
 //   warp 16      owns TMEM and issues the MMAs;
-//   warps 20-27  softmax, two warps per TMEM sub-partition: warps 20+s and 24+s
-//                share the 32 heads (TMEM lanes) of sub-partition s and split
-//                the 64 key columns of a block and the 256 output columns in
-//                halves; they stage Q into TMEM, exchange with the peer CTA,
-//                write P and, at the end, O.
-// setmaxnreg gives the softmax warpgroups 152 registers and the others 40.
+//   warps 20-23  softmax of the CTA's own heads (TMEM lanes 32s .. 32s+15);
+//   warps 24-27  send the peer's partial S (lanes 32s+16 .. 32s+31);
+//   warps 28-31  take in the peer's P rows and rescale factors, rescale the
+//                peer's O rows here, and write those rows at the end.
+// CTA1's 64 rope dims are needed only by QK^T, so they sit in a ring of their
+// own that is released as soon as QK^T has read them.
 #include "dsa_common.cuh"
 #include "dsa_kernels.h"
 
@@ -50,66 +59,152 @@ namespace {
 
 constexpr int kH = 128;              // query heads = MMA M
 constexpr int kBK = 64;              // keys per block = QK^T MMA N
-constexpr int kStages = 4;
-constexpr int kMaxCh = 5;            // 64-dim chunks per CTA (CTA1: 5, CTA0: 4)
+constexpr int kStages = 4;           // ring of the four 64-dim value chunks of a key block
+constexpr int kRopeStages = 2;       // ring of CTA1's rope chunk
 constexpr int kChunkKV = kBK * 128;  // one 64-dim chunk of a key block: 64 rows x 128 B
 constexpr int kMaxK = 2048;
 constexpr int kMaxBlocks = kMaxK / kBK;
-// Warp roles (28 warps, 7 per SM sub-partition). One TMA tile::gather4 request
-// moves four 128-byte row pieces and keeps its issuing warp busy ~90 cycles;
-// measured on B200, the gather rate grows with the number of issuing warps
-// (not lanes), so 19 warps issue them. Registers are moved to the softmax
-// warps with setmaxnreg: 20 warps x 40 + 8 warps x 152 = 896 threads x 72.
+// Warp roles. One TMA tile::gather4 request moves four 128-byte row pieces
+// and keeps its issuing warp busy ~90 cycles; measured on B200, the gather
+// rate grows with the number of issuing warps (not lanes), so 19 warps issue.
 constexpr int kPlanWarps = 16;       // warps 0-15 scan the index row (two blocks each)
 constexpr int kMmaWarp = 16;
 constexpr int kGatherIssuers = 19;   // warps 0-15 and 17-19 issue gather4 requests
-constexpr int kSoftmaxWarp0 = 20;    // warps 20..27
-constexpr int kSoftmaxThreads = 256;
-constexpr int kThreads = (kSoftmaxWarp0 + 8) * 32;
-constexpr uint32_t kRegsSmall = 40;
-constexpr uint32_t kRegsSoftmax = 152;
+constexpr int kSoftmaxWarp0 = 20;    // 20..23
+constexpr int kSendWarp0 = 24;       // 24..27
+constexpr int kRecvWarp0 = 28;       // 28..31
+constexpr int kThreads = 32 * 32;
+// setmaxnreg: the block is launched with 64 registers per thread (65,536);
+// warps 0-19 drop to 48, the softmax warps rise to 128 and the exchange warps
+// to 72: 20 x 48 + 4 x 128 + 8 x 72 = 2048 per 32 threads, all 65,536, and
+// per SM sub-partition 5 x 48 + 128 + 2 x 72 = 512 x 32 = 16,384.
+constexpr uint32_t kRegsSmall = 48;
+constexpr uint32_t kRegsSoftmax = 128;
+constexpr uint32_t kRegsExchange = 72;
 constexpr uint32_t kTmemCols = 512;  // O: [0,256), S: [256,320), Q: [320,480)
 constexpr uint32_t kColO = 0;
 constexpr uint32_t kColS = 256;
 constexpr uint32_t kColQ = 320;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr uint32_t kRxSBytes = 64 * kBK * 4;        // the peer's partial S of our 64 heads
+constexpr uint32_t kRxPBytes = 64 * 128 + 64 * 4;   // the peer's 64 P rows + rescale factors
 
 struct __align__(1024) Smem {
-  uint8_t kv[kStages][kMaxCh][kChunkKV];      // 160 KB key-block ring
-  uint8_t p[kH * 128];                        // 16 KB: P [128 heads x 64 keys] bf16
-  float recv[kH * kBK];                       // 32 KB: peer's partial S
+  uint8_t kv[kStages][4][kChunkKV];           // 128 KB value-chunk ring
+  uint8_t rope[kRopeStages][kChunkKV];        // 16 KB rope-chunk ring (CTA1)
+  uint8_t p[2][kH * 128];                     // 2 x 16 KB: P [128 rows x 64 keys] bf16
+  float rx_s[64 * kBK];                       // 16 KB: the peer's partial S of our heads
+  float tx_s[64 * kBK];                       // 16 KB: our partial S of the peer's heads
   int32_t rows[kMaxK];                        // KV row of every index entry (0 if invalid)
   uint32_t bmask[kMaxBlocks][2];              // valid entries of block b
   uint32_t mask[kMaxBlocks][2];               // valid entries of the j-th non-empty block
   int32_t blk[kMaxBlocks];                    // block number of the j-th non-empty block
-  float red[2][kH][2];                        // per-half row maxima (double buffered by block)
-  float lsum[kH][2];                          // per-half row sums (end of query)
+  __align__(16) float rx_alpha[2][64];        // the peer's rescale factors of its heads
+  __align__(16) float tx_alpha[2][64];        // our rescale factors, copied to the peer
+  float rx_l[64];                             // the peer's final row sums of its heads
   int32_t n_blocks;
+  int32_t gather_n;                           // blocks the gather walks (issuer 0's view)
+  int32_t gather_go[2];                       // issuer 0: stage ready (1) or give up (0)
   uint64_t plan_full, q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t rope_full[kRopeStages], rope_empty[kRopeStages];
   uint64_t s_full, s_empty;
-  uint64_t p_full, p_empty;
+  uint64_t p_full[2], p_empty[2];
   uint64_t o_full;
-  uint64_t rx_full;   // the peer has written its partial into recv
-  uint64_t rx_free;   // the peer has read its own recv (we may write into it)
-  uint64_t pair[4];   // the two softmax warps of sub-partition s have posted red/lsum
+  uint64_t rxs_full;   // the peer's partial S of this block has landed in rx_s
+  uint64_t rxs_free;   // the peer has read its rx_s (we may send the next block)
+  uint64_t rxp_full[2];   // the peer's P rows and factors of a block have landed
+  uint64_t l_full;     // the peer's row sums have landed
   uint32_t tmem_base;
 };
+
+// 2^x with the ex2.approx instruction (flush-to-zero; 2^-inf = 0). P is
+// rounded to bf16 right after, far coarser than the instruction's error.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Maximum of 32 values as a balanced tree (5 dependent steps instead of 32).
+__device__ __forceinline__ float max_tree32(const float (&x)[32]) {
+  float m[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m[i] = fmaxf(x[2 * i], x[2 * i + 1]);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+  return m[0];
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// 16 TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
+// Writes this CTA's 256 O columns of one head per thread pair, scaled by inv,
+// from TMEM lanes (t_lane lane) + (t & 15); thread t covers columns
+// 64c + 32 (t >> 4) .. +31 for c = 0..3. zero: write zeros.
+__device__ __forceinline__ void write_o_rows(uint32_t t_lane, __nv_bfloat16* orow, int hh,
+                                             float inv, bool zero) {
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    uint32_t o[32];
+    tmem_ld16x2_32(t_lane + kColO + 64 * c, o);
+    tmem_wait_ld();
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      pk[i] = pack_bf16x2(zero ? 0.f : __uint_as_float(o[2 * i]) * inv,
+                          zero ? 0.f : __uint_as_float(o[2 * i + 1]) * inv);
+    uint4* dst = reinterpret_cast<uint4*>(orow + 64 * c + 32 * hh);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+  }
+}
+
+// Multiplies the 256 O columns of TMEM lanes (t_lane lane) + (t & 15) by alpha.
+__device__ __forceinline__ void rescale_o_rows(uint32_t t_lane, float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    uint32_t o[32];
+    tmem_ld16x2_32(t_lane + kColO + 64 * c, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+    tmem_st16x2_32(t_lane + kColO + 64 * c, o);
+  }
+  tmem_wait_st();
+}
+
+// Stages 64-dim chunks cs[] (those below nch) of this thread's Q row into
+// TMEM columns 32 c of taddr_q, all loads issued before the first store.
+template <int N>
+__device__ __forceinline__ void stage_q_chunks(uint32_t taddr_q, const uint4* src,
+                                               const int (&cs)[N], int nch) {
+  uint4 qv[8 * N];
+#pragma unroll
+  for (int k = 0; k < N; ++k)
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      qv[8 * k + i] = cs[k] < nch ? __ldg(src + cs[k] * 8 + i) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    if (cs[k] < nch) {
+      uint32_t w[32];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        w[4 * i + 0] = qv[8 * k + i].x;
+        w[4 * i + 1] = qv[8 * k + i].y;
+        w[4 * i + 2] = qv[8 * k + i].z;
+        w[4 * i + 3] = qv[8 * k + i].w;
+      }
+      tmem_st32(taddr_q + 32 * cs[k], w);
+    }
+  }
+  tmem_wait_st();
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -138,19 +233,26 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
 
   if (threadIdx.x == 0) {
     mbar_init(&S.plan_full, 1);
-    mbar_init(&S.q_full, kSoftmaxThreads);
+    mbar_init(&S.q_full, 3 * 128);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&S.kv_full[i], 1);   // the expect-tx arrival; gather4 bytes complete it
       mbar_init(&S.kv_empty[i], 1);
     }
+    for (int i = 0; i < kRopeStages; ++i) {
+      mbar_init(&S.rope_full[i], 1);
+      mbar_init(&S.rope_empty[i], 1);
+    }
     mbar_init(&S.s_full, 1);
-    mbar_init(&S.s_empty, kSoftmaxThreads);
-    mbar_init(&S.p_full, kSoftmaxThreads);
-    mbar_init(&S.p_empty, 1);
+    mbar_init(&S.s_empty, 2 * 128);   // softmax and send warps
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.p_full[b], 2 * 128);    // softmax and receive warps
+      mbar_init(&S.p_empty[b], 2);         // this CTA's PV and the peer's PV are done
+      mbar_init(&S.rxp_full[b], 1);
+    }
     mbar_init(&S.o_full, 1);
-    mbar_init(&S.rx_full, 1);    // one expect-tx arrival; the peer's st.async bytes complete it
-    mbar_init(&S.rx_free, 8);    // one arrival per peer softmax warp
-    for (int i = 0; i < 4; ++i) mbar_init(&S.pair[i], 64);
+    mbar_init(&S.rxs_full, 1);        // one expect-tx arrival; the peer's st.async bytes
+    mbar_init(&S.rxs_free, 4);        // one arrival per peer softmax warp
+    mbar_init(&S.l_full, 1);
     fence_barrier_init();
     if (!q_ok) report(a.status, DSA_ERR_DEVICE_BOUNDS);
   }
@@ -162,343 +264,435 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
   const uint32_t tmem_base = S.tmem_base;
 
   if (warp < kSoftmaxWarp0) {
-  regs_dec<kRegsSmall>();
-  if (warp < kPlanWarps) {
-    // ------------------------------------------------------------ plan (warps 0-15)
-    const int32_t* irow = a.idx + static_cast<int64_t>(qi) * a.ld_idx;
-    // warp w scans blocks 2w and 2w+1; e[2i + half] holds entry
-    // (2w + i) * 64 + 32 half + lane
-    int e[4];
-    bool bad = false;
+    regs_dec<kRegsSmall>();
+    if (warp < kPlanWarps) {
+      // ---------------------------------------------------------- plan (warps 0-15)
+      const int32_t* irow = a.idx + static_cast<int64_t>(qi) * a.ld_idx;
+      // warp w scans blocks 2w and 2w+1; e[2i + half] holds entry
+      // (2w + i) * 64 + 32 half + lane
+      int e[4];
+      bool bad = false;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int b = 2 * warp + (i >> 1);
-      const int jj = b * kBK + (i & 1) * 32 + lane;
-      e[i] = (b < nb && jj < a.k) ? __ldg(irow + jj) : -1;
-      bad |= e[i] > pos;
-      e[i] = (e[i] >= 0 && e[i] <= pos) ? e[i] : -1;
-    }
-    int pg[4];
+      for (int i = 0; i < 4; ++i) {
+        const int b = 2 * warp + (i >> 1);
+        const int jj = b * kBK + (i & 1) * 32 + lane;
+        e[i] = (b < nb && jj < a.k) ? __ldg(irow + jj) : -1;
+        bad |= e[i] > pos;
+        e[i] = (e[i] >= 0 && e[i] <= pos) ? e[i] : -1;
+      }
+      int pg[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      pg[i] = (a.keys.paged && e[i] >= 0)
-                  ? __ldg(a.keys.block_table + static_cast<int64_t>(qi) * a.keys.ld_block_table +
-                          (e[i] >> 6))
-                  : 0;
+      for (int i = 0; i < 4; ++i)
+        pg[i] = (a.keys.paged && e[i] >= 0)
+                    ? __ldg(a.keys.block_table +
+                            static_cast<int64_t>(qi) * a.keys.ld_block_table + (e[i] >> 6))
+                    : 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int r = 0;
-      if (e[i] >= 0) {
-        if (!a.keys.paged) {
-          r = e[i];
-        } else if (pg[i] < 0 || pg[i] >= a.keys.num_pages) {
-          bad = true;
-          e[i] = -1;      // an unusable page: skip the entry
-        } else {
-          r = pg[i] * 64 + (e[i] & 63);
+      for (int i = 0; i < 4; ++i) {
+        int r = 0;
+        if (e[i] >= 0) {
+          if (!a.keys.paged) {
+            r = e[i];
+          } else if (pg[i] < 0 || pg[i] >= a.keys.num_pages) {
+            bad = true;
+            e[i] = -1;      // an unusable page: skip the entry
+          } else {
+            r = pg[i] * 64 + (e[i] & 63);
+          }
+        }
+        S.rows[(2 * warp + (i >> 1)) * kBK + (i & 1) * 32 + lane] = r;
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t m0 = __ballot_sync(0xffffffffu, e[2 * i] >= 0);
+        const uint32_t m1 = __ballot_sync(0xffffffffu, e[2 * i + 1] >= 0);
+        if (lane == 0) {
+          S.bmask[2 * warp + i][0] = m0;
+          S.bmask[2 * warp + i][1] = m1;
         }
       }
-      S.rows[(2 * warp + (i >> 1)) * kBK + (i & 1) * 32 + lane] = r;
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const uint32_t m0 = __ballot_sync(0xffffffffu, e[2 * i] >= 0);
-      const uint32_t m1 = __ballot_sync(0xffffffffu, e[2 * i + 1] >= 0);
-      if (lane == 0) {
-        S.bmask[2 * warp + i][0] = m0;
-        S.bmask[2 * warp + i][1] = m1;
-      }
-    }
-    if (rank == 0 && __any_sync(0xffffffffu, bad) && lane == 0)
-      report(a.status, DSA_ERR_DEVICE_BOUNDS);
-    named_bar_sync(1, kPlanWarps * 32);
-    if (threadIdx.x == 0) {
-      int nvb = 0;
-      for (int b = 0; b < nb; ++b) {
-        const uint32_t m0 = S.bmask[b][0], m1 = S.bmask[b][1];
-        if ((m0 | m1) != 0u) {
-          S.mask[nvb][0] = m0;
-          S.mask[nvb][1] = m1;
-          S.blk[nvb] = b;
-          ++nvb;
+      if (rank == 0 && __any_sync(0xffffffffu, bad) && lane == 0)
+        report(a.status, DSA_ERR_DEVICE_BOUNDS);
+      named_bar_sync(1, kPlanWarps * 32);
+      if (threadIdx.x == 0) {
+        int nvb = 0;
+        for (int b = 0; b < nb; ++b) {
+          const uint32_t m0 = S.bmask[b][0], m1 = S.bmask[b][1];
+          if ((m0 | m1) != 0u) {
+            S.mask[nvb][0] = m0;
+            S.mask[nvb][1] = m1;
+            S.blk[nvb] = b;
+            ++nvb;
+          }
         }
+        S.n_blocks = nvb;
+        mbar_arrive(&S.plan_full);
       }
-      S.n_blocks = nvb;
-      mbar_arrive(&S.plan_full);
     }
-  }
-  if (warp != kMmaWarp) {
-    // ------------------------------------------------------------ gather (19 issuing warps)
-    // Block j's 16 groups of 4 rows x nch 64-dim chunks are split over the
-    // issuers: issuer i requests pieces p = i, i + 19, ... (group p / nch,
-    // chunk p % nch), each landing as 4 swizzled 128-byte rows of the stage.
-    const int issuer = warp < kMmaWarp ? warp : warp - 1;
-    if (lane == 0) {
-      bool ok = mbar_wait(&S.plan_full, 0, a.status);
-      const int n = ok ? S.n_blocks : 0;
+    if (warp != kMmaWarp) {
+      // ---------------------------------------------------------- gather (19 issuing warps)
+      // Block j's 16 groups of 4 rows x nch 64-dim chunks are split over the
+      // issuers: issuer i requests pieces p = i, i + 19, ... (group p / nch,
+      // chunk p % nch), each landing as 4 swizzled 128-byte rows; chunk 4
+      // (CTA1's rope dims) goes to the rope ring.
+      // Only issuer 0 waits on the ring's barriers; the other 18 warps sleep on
+      // hardware named barrier 2 (taking no issue slots from the softmax warps)
+      // and learn from a shared flag whether to go on, so all 19 always take
+      // the same number of barrier steps.
+      const int issuer = warp < kMmaWarp ? warp : warp - 1;
+      if (issuer == 0) {
+        const bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
+        if (lane == 0) S.gather_n = ok ? S.n_blocks : 0;
+      }
+      named_bar_sync(2, kGatherIssuers * 32);
+      const int n = S.gather_n;
       const int n_req = (kBK / 4) * nch;
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
-        const uint32_t ph = static_cast<uint32_t>(j / kStages) & 1u;
-        if (!mbar_wait(&S.kv_empty[st], ph ^ 1u, a.status)) break;
-        if (issuer == 0) mbar_arrive_expect_tx(&S.kv_full[st], nch * kChunkKV);
-        const int* rb = S.rows + S.blk[j] * kBK;
-        for (int p = issuer; p < n_req; p += kGatherIssuers) {
-          const int g = p / nch, c = p - g * nch;
-          const int4 r4 = *reinterpret_cast<const int4*>(rb + 4 * g);
-          tma_gather4(S.kv[st][c] + g * 512, &a.map_kv, col0 + 64 * c, r4.x, r4.y, r4.z, r4.w,
-                      &S.kv_full[st]);
-        }
-      }
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    const uint32_t idesc_qk = make_idesc(kBK, 1, 1, 0, 0);   // bf16, A (TMEM) and B K-major
-    const uint32_t idesc_pv = make_idesc(256, 1, 1, 0, 1);   // bf16, K-major P, MN-major V
-    const uint64_t pdesc = sw128_desc(smem_u32(S.p), 16, 1024);
-    bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
-    const int n = ok ? S.n_blocks : 0;
-    ok = ok && mbar_wait_warp(&S.q_full, 0, a.status);
-    tc_fence_after();
-    auto issue_pv = [&](int pst, int jj) -> bool {
-      if (!mbar_wait_warp(&S.p_full, static_cast<uint32_t>(jj & 1), a.status)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint64_t vdesc = sw128_desc(smem_u32(S.kv[pst][0]), kChunkKV, 1024);
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk)
-          mma_bf16(tmem_base + kColO, pdesc + 2 * kk, vdesc + 128 * kk, idesc_pv,
-                   (jj > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&S.kv_empty[pst]);
-        mma_commit(&S.p_empty);
-      }
-      __syncwarp();
-      return true;
-    };
-    int j = 0, prev_st = 0;
-    for (; j < n && ok; ++j) {
-      const int st = j % kStages;
-      const uint32_t ph = static_cast<uint32_t>(j / kStages) & 1u;
-      if (!mbar_wait_warp(&S.kv_full[st], ph, a.status) ||
-          !mbar_wait_warp(&S.s_empty, static_cast<uint32_t>((j & 1) ^ 1), a.status)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t d = tmem_base + kColS;
-        for (int c = 0; c < nch; ++c) {
-          const uint64_t kd = sw128_desc(smem_u32(S.kv[st][c]), 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ts(d, tmem_base + kColQ + c * 32 + kk * 8, kd + 2 * kk, idesc_qk,
-                        (c | kk) != 0 ? 1u : 0u);
-        }
-        mma_commit(&S.s_full);
-      }
-      __syncwarp();
-      if (j > 0 && !issue_pv(prev_st, j - 1)) {
-        ok = false;
-        break;
-      }
-      prev_st = st;
-    }
-    if (ok && n > 0) issue_pv(prev_st, n - 1);
-    if (lane == 0) mma_commit(&S.o_full);
-  }
-  } else {
-    regs_inc<kRegsSoftmax>();
-    // ------------------------------------------------------------ softmax (warps 20-27)
-    const int sub = warp & 3;                              // TMEM sub-partition
-    const int hf = (warp - kSoftmaxWarp0) >> 2;            // column half of this warp
-    const int h = sub * 32 + lane;                         // head = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-    uint64_t* pair_bar = &S.pair[sub];   // both warps of the sub-partition, 64 arrivals per use
-    {
-      // Q -> TMEM: this CTA's slice of q[t, h, :] as raw bf16 pairs; the two
-      // warps of a sub-partition stage alternate 64-dim chunks
-      const uint4* src = reinterpret_cast<const uint4*>(
-          a.q + static_cast<int64_t>(qi) * a.ld_q + static_cast<int64_t>(h) * 576 + col0);
-      uint4 qv[24];
-#pragma unroll
-      for (int i = 0; i < 24; ++i) {
-        const int c = hf + 2 * (i >> 3);        // chunks hf, hf+2, hf+4
-        qv[i] = c < nch ? __ldg(src + c * 8 + (i & 7)) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int cc = 0; cc < 3; ++cc) {
-        const int c = hf + 2 * cc;
-        if (c < nch) {
-          uint32_t w[32];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            w[4 * i + 0] = qv[cc * 8 + i].x;
-            w[4 * i + 1] = qv[cc * 8 + i].y;
-            w[4 * i + 2] = qv[cc * 8 + i].z;
-            w[4 * i + 3] = qv[cc * 8 + i].w;
+        const int rs = j % kRopeStages;
+        if (issuer == 0) {
+          bool ok = mbar_wait_warp(&S.kv_empty[st], static_cast<uint32_t>((j / kStages) & 1) ^ 1u,
+                                   a.status);
+          if (ok && rank == 1)
+            ok = mbar_wait_warp(&S.rope_empty[rs],
+                                static_cast<uint32_t>((j / kRopeStages) & 1) ^ 1u, a.status);
+          if (lane == 0) {
+            if (ok) {
+              mbar_arrive_expect_tx(&S.kv_full[st], 4 * kChunkKV);
+              if (rank == 1) mbar_arrive_expect_tx(&S.rope_full[rs], kChunkKV);
+            }
+            S.gather_go[j & 1] = ok ? 1 : 0;
           }
-          tmem_st32(tmem_base + lane_off + kColQ + 32 * c, w);
         }
+        named_bar_sync(2, kGatherIssuers * 32);
+        if (S.gather_go[j & 1] == 0) break;
+        if (lane == 0) {
+          const int* rb = S.rows + S.blk[j] * kBK;
+          for (int p = issuer; p < n_req; p += kGatherIssuers) {
+            const int g = p / nch, c = p - g * nch;
+            const int4 r4 = *reinterpret_cast<const int4*>(rb + 4 * g);
+            if (c < 4)
+              tma_gather4(S.kv[st][c] + g * 512, &a.map_kv, col0 + 64 * c, r4.x, r4.y, r4.z,
+                          r4.w, &S.kv_full[st]);
+            else
+              tma_gather4(S.rope[rs] + g * 512, &a.map_kv, 512, r4.x, r4.y, r4.z, r4.w,
+                          &S.rope_full[rs]);
+          }
+        }
+        __syncwarp();
       }
-      tmem_wait_st();
+    } else {
+      // ---------------------------------------------------------- MMA issuer
+      const uint32_t idesc_qk = make_idesc(kBK, 1, 1, 0, 0);   // bf16, A (TMEM) and B K-major
+      const uint32_t idesc_pv = make_idesc(256, 1, 1, 0, 1);   // bf16, K-major P, MN-major V
+      bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
+      const int n = ok ? S.n_blocks : 0;
+      ok = ok && mbar_wait_warp(&S.q_full, 0, a.status);
+      tc_fence_after();
+      // QK^T of block jj into S once the softmax and send warps have read S_{jj-1}
+      auto issue_qk = [&](int jj) -> bool {
+        const int st = jj % kStages;
+        const int rs = jj % kRopeStages;
+        if (!mbar_wait_warp(&S.kv_full[st], static_cast<uint32_t>(jj / kStages) & 1u,
+                            a.status))
+          return false;
+        if (rank == 1 &&
+            !mbar_wait_warp(&S.rope_full[rs], static_cast<uint32_t>(jj / kRopeStages) & 1u,
+                            a.status))
+          return false;
+        if (!mbar_wait_warp(&S.s_empty, static_cast<uint32_t>((jj & 1) ^ 1), a.status))
+          return false;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t d = tmem_base + kColS;
+          for (int c = 0; c < nch; ++c) {
+            const uint64_t kd =
+                sw128_desc(smem_u32(c < 4 ? S.kv[st][c] : S.rope[rs]), 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ts(d, tmem_base + kColQ + c * 32 + kk * 8, kd + 2 * kk, idesc_qk,
+                          (c | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&S.s_full);
+          if (rank == 1) mma_commit(&S.rope_empty[rs]);
+        }
+        __syncwarp();
+        return true;
+      };
+      // O += P V of block jj once every P row of it is in place
+      auto issue_pv = [&](int jj) -> bool {
+        const int b = jj & 1;
+        if (!mbar_wait_warp(&S.p_full[b], static_cast<uint32_t>(jj >> 1) & 1u, a.status))
+          return false;
+        tc_fence_after();
+        if (lane == 0) {
+          const int st = jj % kStages;
+          const uint64_t pdesc = sw128_desc(smem_u32(S.p[b]), 16, 1024);
+          const uint64_t vdesc = sw128_desc(smem_u32(S.kv[st][0]), kChunkKV, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_bf16(tmem_base + kColO, pdesc + 2 * kk, vdesc + 128 * kk, idesc_pv,
+                     (jj > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&S.kv_empty[st]);
+          mma_commit(&S.p_empty[b]);
+          // the peer may overwrite its rows of this P tile
+          mma_commit_cluster(mapa_shared(smem_u32(&S.p_empty[b]), peer));
+        }
+        __syncwarp();
+        return true;
+      };
+      ok = ok && (n == 0 || issue_qk(0));
+      for (int j = 0; j < n && ok; ++j) {
+        if (j + 1 < n && !issue_qk(j + 1)) ok = false;
+        if (ok && !issue_pv(j)) ok = false;
+      }
+      if (lane == 0) mma_commit(&S.o_full);
+    }
+  } else if (warp < kSendWarp0) {
+    regs_inc<kRegsSoftmax>();
+    const int s = warp & 3;                     // TMEM sub-partition
+    const int i16 = lane & 15;
+    const int hh = lane >> 4;                   // key half (S) / column half (O)
+    const int o = 16 * s + i16;                 // index among the owner's 64 heads
+    const uint32_t sw = static_cast<uint32_t>(i16 & 7);
+    const uint32_t lane_q = static_cast<uint32_t>(32 * s) << 16;
+    // Q -> TMEM (32x32b: thread = lane 32s + lane). Row order: lane 32s+i is
+    // own head 64 rank + 16s + i, lane 32s+16+i the peer's head.
+    const uint4* qsrc = reinterpret_cast<const uint4*>(
+        a.q + static_cast<int64_t>(qi) * a.ld_q +
+        static_cast<int64_t>(64 * static_cast<int>(rank ^ static_cast<uint32_t>(lane >> 4)) +
+                             16 * s + (lane & 15)) * 576 +
+        col0);
+    {
+      const int cs[3] = {0, 3, 4};   // the send and receive warps stage 1 and 2
+      stage_q_chunks(tmem_base + lane_q + kColQ, qsrc, cs, nch);
       tc_fence_before();
       mbar_arrive(&S.q_full);
     }
-    // this warp's 16-byte chunks of row h of the exchange buffer: 8*hf .. 8*hf+7
-    const uint32_t sw = static_cast<uint32_t>(h & 7);
-    const uint32_t recv_row = smem_u32(S.recv) + static_cast<uint32_t>(h) * 256u;
-    const uint32_t recv_peer = mapa_shared(recv_row, peer);
-    const uint32_t rx_full_peer = mapa_shared(smem_u32(&S.rx_full), peer);
-    const uint32_t rx_free_peer = mapa_shared(smem_u32(&S.rx_free), peer);
-    uint8_t* prow = S.p + (h >> 3) * 1024 + (h & 7) * 128;
-    const float sl2 = a.scale_log2;
-    float m_used = -INFINITY, l = 0.f;
     bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
     const int n = ok ? S.n_blocks : 0;
-    int j = 0;
-    for (; j < n && ok; ++j) {
-      const uint32_t mk = S.mask[j][hf];          // valid keys among this warp's 32 columns
-      // own partial S for this warp's columns
-      if (!mbar_wait_warp(&S.s_full, static_cast<uint32_t>(j & 1), a.status)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t v[32];
-      {
-        uint32_t (&v0)[16] = *reinterpret_cast<uint32_t(*)[16]>(&v[0]);
-        uint32_t (&v1)[16] = *reinterpret_cast<uint32_t(*)[16]>(&v[16]);
-        tmem_ld16(tmem_base + lane_off + kColS + 32 * hf, v0);
-        tmem_ld16(tmem_base + lane_off + kColS + 32 * hf + 16, v1);
-        tmem_wait_ld();
-      }
-      tc_fence_before();
-      mbar_arrive(&S.s_empty);
-      // this block's expected bytes from the peer (all 32 KB of it)
-      if (h == 0 && hf == 0) mbar_arrive_expect_tx(&S.rx_full, kH * kBK * 4);
-      // send ours once the peer has consumed the previous block
-      if (!mbar_wait_cluster_warp(&S.rx_free, static_cast<uint32_t>((j & 1) ^ 1), a.status)) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t cc = (static_cast<uint32_t>(8 * hf + c) ^ sw) << 4;
-        st_async_v4(recv_peer + cc, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3],
-                    rx_full_peer);
-      }
-      // receive the peer's partial and add (fp32 addition is commutative:
-      // both CTAs get identical S)
-      if (!mbar_wait_cluster_warp(&S.rx_full, static_cast<uint32_t>(j & 1), a.status)) {
-        ok = false;
-        break;
-      }
-      float x[32];
-      const float4* rp = reinterpret_cast<const float4*>(S.recv + h * kBK);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float4 pv = rp[(8 * hf + c) ^ static_cast<int>(sw)];
-        x[4 * c + 0] = __uint_as_float(v[4 * c + 0]) + pv.x;
-        x[4 * c + 1] = __uint_as_float(v[4 * c + 1]) + pv.y;
-        x[4 * c + 2] = __uint_as_float(v[4 * c + 2]) + pv.z;
-        x[4 * c + 3] = __uint_as_float(v[4 * c + 3]) + pv.w;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster_relaxed(rx_free_peer);   // values already consumed
-      // row max of this half (masked), combined with the other half
-      float bm = -INFINITY;
-      if (mk == 0xffffffffu) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) bm = fmaxf(bm, x[i]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          x[i] = ((mk >> i) & 1u) ? x[i] : -INFINITY;
-          bm = fmaxf(bm, x[i]);
+    {
+      // ---------------------------------------------------------- softmax of own heads
+      // thread t: head 64 rank + o in TMEM lane 32s + (t & 15), keys 32 hh .. +31
+      const int head = 64 * static_cast<int>(rank) + o;
+      const uint32_t t_lane = tmem_base + lane_q;
+      const uint32_t m_own = static_cast<uint32_t>(32 * s + i16);   // our P row of the head
+      const uint32_t prow_off = (m_own >> 3) * 1024 + (m_own & 7) * 128;
+      // this warp's 16 P rows 32s .. 32s+15 are bytes [4096 s, +2048) of a P
+      // tile; in the peer they are rows 32s+16 .. 32s+31, bytes [4096 s + 2048, +2048)
+      const uint32_t p_peer0 = mapa_shared(smem_u32(S.p[0]), peer) + 4096u * s + 2048u;
+      const uint32_t rxp_full_peer0 = mapa_shared(smem_u32(&S.rxp_full[0]), peer);
+      const uint32_t alpha_peer0 = mapa_shared(smem_u32(&S.rx_alpha[0][16 * s]), peer);
+      const uint32_t rxs_free_peer = mapa_shared(smem_u32(&S.rxs_free), peer);
+      const float sl2 = a.scale_log2;
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < n && ok; ++j) {
+        const int b = j & 1;                       // P tile of this block
+        const uint32_t mk = S.mask[j][hh];         // valid keys among this thread's 32
+        // own partial S of the block
+        if (!mbar_wait_warp(&S.s_full, static_cast<uint32_t>(j & 1), a.status)) {
+          ok = false;
+          break;
         }
-      }
-      S.red[j & 1][h][hf] = bm;
-      mbar_arrive(pair_bar);
-      if (!mbar_wait_warp(pair_bar, static_cast<uint32_t>(j & 1), a.status)) {
-        ok = false;
-        break;
-      }
-      bm = fmaxf(bm, S.red[j & 1][h][hf ^ 1]) * sl2;   // scale > 0: max commutes with it
-      const float m_new = fmaxf(m_used, bm);
-      const bool rescale = m_new > m_used + kRescaleLog2;
-      const float m_next = rescale ? m_new : m_used;
-      const float alpha = rescale ? exp2f(m_used - m_next) : 1.f;
-      // previous PV done: P buffer free, O stable
-      if (!mbar_wait_warp(&S.p_empty, static_cast<uint32_t>((j & 1) ^ 1), a.status)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-        // this warp's 128 of the 256 output columns
-#pragma unroll 1
+        tc_fence_after();
+        uint32_t v[32];
+        tmem_ld16x2_32(t_lane + kColS, v);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&S.s_empty);
+        // the peer's partial for our heads
+        if (warp == kSoftmaxWarp0 && lane == 0) mbar_arrive_expect_tx(&S.rxs_full, kRxSBytes);
+        if (!mbar_wait_cluster_warp(&S.rxs_full, static_cast<uint32_t>(j & 1), a.status)) {
+          ok = false;
+          break;
+        }
+        float x[32];
+        const float4* rp = reinterpret_cast<const float4*>(S.rx_s + o * kBK);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float4 pv = rp[(8 * hh + c) ^ static_cast<int>(sw)];
+          x[4 * c + 0] = __uint_as_float(v[4 * c + 0]) + pv.x;
+          x[4 * c + 1] = __uint_as_float(v[4 * c + 1]) + pv.y;
+          x[4 * c + 2] = __uint_as_float(v[4 * c + 2]) + pv.z;
+          x[4 * c + 3] = __uint_as_float(v[4 * c + 3]) + pv.w;
+        }
+        // release: the loads above are ordered before the peer's next writes.
+        // Lane 31 arrives: lane 0 issues the bulk copies, which a release by it
+        // would wait on.
+        __syncwarp();
+        if (lane == 31) mbar_arrive_cluster(rxs_free_peer);
+        // block row max over both key halves (threads t and t ^ 16 share a head)
+        if (mk != 0xffffffffu) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = ((mk >> i) & 1u) ? x[i] : -INFINITY;
+        }
+        float bm = max_tree32(x);
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16)) * sl2;   // scale > 0
+        const float m_new = fmaxf(m_used, bm);
+        const bool rescale = m_new > m_used + kRescaleLog2;
+        const float m_next = rescale ? m_new : m_used;
+        const float alpha = rescale ? fast_exp2(m_used - m_next) : 1.f;
+        // PV of block j-2 done in both CTAs: P tile b free here and in the peer
+        if (!mbar_wait_cluster_warp(&S.p_empty[b], static_cast<uint32_t>((j >> 1) & 1) ^ 1u,
+                                    a.status)) {
+          ok = false;
+          break;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+          // O stable: PV of block j-1 done
+          if (!mbar_wait_cluster_warp(&S.p_empty[b ^ 1],
+                                      static_cast<uint32_t>((j - 1) >> 1) & 1u, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          rescale_o_rows(t_lane, alpha);
+        }
+        if (hh == 0) S.tx_alpha[b][o] = alpha;
+        uint8_t* prow = S.p[b] + prow_off;
+        l *= alpha;
+        m_used = m_next;
+        const float neg_m = -m_used;
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          const uint32_t col = kColO + 128 * hf + 32 * c;
-          tmem_ld32(tmem_base + lane_off + col, o);
-          tmem_wait_ld();
+          uint32_t w4[4];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem_base + lane_off + col, o);
+          for (int i = 0; i < 4; ++i) {
+            const float p0 = fast_exp2(fmaf(x[8 * c + 2 * i], sl2, neg_m));
+            const float p1 = fast_exp2(fmaf(x[8 * c + 2 * i + 1], sl2, neg_m));
+            ps[i] += p0 + p1;
+            w4[i] = pack_bf16x2(p0, p1);
+          }
+          const uint32_t cc = (static_cast<uint32_t>(4 * hh + c) ^ sw) << 4;
+          *reinterpret_cast<uint4*>(prow + cc) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
-        tmem_wait_st();
-      }
-      l *= alpha;
-      m_used = m_next;
-      const float neg_m = -m_used;
-      float psum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t w4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float p0 = exp2f(fmaf(x[8 * c + 2 * i], sl2, neg_m));
-          const float p1 = exp2f(fmaf(x[8 * c + 2 * i + 1], sl2, neg_m));
-          psum += p0 + p1;
-          w4[i] = pack_bf16x2(p0, p1);
+        l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+        // P rows and factors visible to the async proxy (our MMA, the copy to the peer)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t bb = static_cast<uint32_t>(b);
+          const uint32_t rxp_full_peer = rxp_full_peer0 + 8u * bb;
+          bulk_copy_to_cluster(p_peer0 + bb * (kH * 128), smem_u32(S.p[b]) + 4096u * s, 2048,
+                               rxp_full_peer);
+          bulk_copy_to_cluster(alpha_peer0 + 256u * bb, smem_u32(&S.tx_alpha[b][16 * s]), 64,
+                               rxp_full_peer);
         }
-        *reinterpret_cast<uint4*>(prow + ((static_cast<uint32_t>(4 * hf + c) ^ sw) << 4)) =
-            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        tc_fence_before();
+        mbar_arrive(&S.p_full[b]);
       }
-      l += psum;
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&S.p_full);
+      // epilogue: O / l -> bf16 for own heads, lse; the peer gets l for its rows
+      const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      if (hh == 0)
+        st_async_b32(mapa_shared(smem_u32(&S.rx_l[o]), peer), __float_as_uint(lt),
+                     mapa_shared(smem_u32(&S.l_full), peer));
+      if (mbar_wait_warp(&S.o_full, 0, a.status)) {
+        tc_fence_after();
+        const bool zero = !ok || n == 0 || !(lt > 0.f);
+        write_o_rows(t_lane, a.out + (static_cast<int64_t>(qi) * kH + head) * 512 + col0, hh,
+                     zero ? 0.f : 1.f / lt, zero);
+        if (hh == 0 && a.lse != nullptr)
+          a.lse[static_cast<int64_t>(qi) * kH + head] =
+              zero ? -INFINITY : (m_used + log2f(lt)) * 0.69314718055994531f;
+      }
     }
-    // epilogue: O / l -> bf16, lse (l summed over both halves)
-    S.lsum[h][hf] = l;
-    mbar_arrive(pair_bar);
-    const bool pair_ok = mbar_wait_warp(pair_bar, static_cast<uint32_t>(j & 1), a.status);
-    ok = ok && pair_ok;
-    const float lt = S.lsum[h][0] + S.lsum[h][1];
-    if (mbar_wait_warp(&S.o_full, 0, a.status)) {
-      tc_fence_after();
-      const float inv = (ok && lt > 0.f) ? 1.f / lt : 0.f;
-      __nv_bfloat16* orow = a.out + (static_cast<int64_t>(qi) * kH + h) * 512 +
-                            static_cast<int64_t>(col0 + 128 * hf);
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tmem_base + lane_off + kColO + 128 * hf + 32 * c, o);
+  } else {
+    regs_inc<kRegsExchange>();
+    const int s = warp & 3;                     // TMEM sub-partition
+    const int i16 = lane & 15;
+    const int hh = lane >> 4;                   // key half (S) / column half (O)
+    const int o = 16 * s + i16;                 // index among the owner's 64 heads
+    const uint32_t sw = static_cast<uint32_t>(i16 & 7);
+    const uint32_t lane_q = static_cast<uint32_t>(32 * s) << 16;
+    // Q -> TMEM (32x32b: thread = lane 32s + lane). Row order: lane 32s+i is
+    // own head 64 rank + 16s + i, lane 32s+16+i the peer's head.
+    const uint4* qsrc = reinterpret_cast<const uint4*>(
+        a.q + static_cast<int64_t>(qi) * a.ld_q +
+        static_cast<int64_t>(64 * static_cast<int>(rank ^ static_cast<uint32_t>(lane >> 4)) +
+                             16 * s + (lane & 15)) * 576 +
+        col0);
+    {
+      const int cs[1] = {warp < kRecvWarp0 ? 1 : 2};
+      stage_q_chunks(tmem_base + lane_q + kColQ, qsrc, cs, nch);
+      tc_fence_before();
+      mbar_arrive(&S.q_full);
+    }
+    bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
+    const int n = ok ? S.n_blocks : 0;
+    if (warp < kRecvWarp0) {
+      // ---------------------------------------------------------- send the peer's partial S
+      // thread t: the peer's head o in TMEM lane 32s + 16 + (t & 15), keys 32 hh .. +31
+      const uint32_t t_lane = tmem_base + lane_q + (16u << 16);
+      uint8_t* tx_row = reinterpret_cast<uint8_t*>(S.tx_s + o * kBK);
+      // this warp's rows 16s .. 16s+15 of tx_s go to the same rows of the peer's rx_s
+      const uint32_t tx_warp = smem_u32(S.tx_s + 16 * s * kBK);
+      const uint32_t rxs_peer_warp = mapa_shared(smem_u32(S.rx_s + 16 * s * kBK), peer);
+      const uint32_t rxs_full_peer = mapa_shared(smem_u32(&S.rxs_full), peer);
+      for (int j = 0; j < n && ok; ++j) {
+        if (!mbar_wait_warp(&S.s_full, static_cast<uint32_t>(j & 1), a.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t v[32];
+        tmem_ld16x2_32(t_lane + kColS, v);
         tmem_wait_ld();
-        uint32_t pk[16];
+        tc_fence_before();
+        mbar_arrive(&S.s_empty);
+        // the peer has read block j-1 out of its rx_s (so our copy out of tx_s is done)
+        if (!mbar_wait_cluster_warp(&S.rxs_free, static_cast<uint32_t>((j & 1) ^ 1),
+                                    a.status)) {
+          ok = false;
+          break;
+        }
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(j > 0 ? __uint_as_float(o[2 * i]) * inv : 0.f,
-                              j > 0 ? __uint_as_float(o[2 * i + 1]) * inv : 0.f);
-        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t cc = (static_cast<uint32_t>(8 * hh + c) ^ sw) << 4;
+          *reinterpret_cast<uint4*>(tx_row + cc) = make_uint4(v[4 * c], v[4 * c + 1],
+                                                              v[4 * c + 2], v[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) bulk_copy_to_cluster(rxs_peer_warp, tx_warp, 16 * kBK * 4, rxs_full_peer);
       }
-      if (rank == 0 && hf == 0 && a.lse != nullptr)
-        a.lse[static_cast<int64_t>(qi) * kH + h] =
-            (ok && lt > 0.f) ? (m_used + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+    } else {
+      // ---------------------------------------------------------- the peer's P rows
+      // thread t: the peer's head in TMEM lane 32s + 16 + (t & 15)
+      const int head = 64 * static_cast<int>(peer) + o;
+      const uint32_t t_lane = tmem_base + lane_q + (16u << 16);
+      for (int j = 0; j < n && ok; ++j) {
+        const int b = j & 1;
+        if (warp == kRecvWarp0 && lane == 0) mbar_arrive_expect_tx(&S.rxp_full[b], kRxPBytes);
+        if (!mbar_wait_cluster_warp(&S.rxp_full[b], static_cast<uint32_t>(j >> 1) & 1u,
+                                    a.status)) {
+          ok = false;
+          break;
+        }
+        const float alpha = S.rx_alpha[b][o];
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // O stable: PV of block j-1 done
+          if (!mbar_wait_cluster_warp(&S.p_empty[b ^ 1],
+                                      static_cast<uint32_t>((j - 1) >> 1) & 1u, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          rescale_o_rows(t_lane, alpha);
+        }
+        fence_proxy_async_smem();   // the peer's rows, seen here, before the MMA reads them
+        tc_fence_before();
+        mbar_arrive(&S.p_full[b]);
+      }
+      if (warp == kRecvWarp0 && lane == 0) mbar_arrive_expect_tx(&S.l_full, 64 * 4);
+      const bool l_ok = mbar_wait_cluster_warp(&S.l_full, 0, a.status);
+      const float lt = l_ok ? S.rx_l[o] : 0.f;
+      if (mbar_wait_warp(&S.o_full, 0, a.status)) {
+        tc_fence_after();
+        const bool zero = !ok || !l_ok || n == 0 || !(lt > 0.f);
+        write_o_rows(t_lane, a.out + (static_cast<int64_t>(qi) * kH + head) * 512 + col0, hh,
+                     zero ? 0.f : 1.f / lt, zero);
+      }
     }
   }
 
