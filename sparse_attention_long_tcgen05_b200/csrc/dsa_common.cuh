@@ -188,6 +188,16 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint3
       : "memory");
 }
 
+// Relaxed arrive on an mbarrier that may live in the peer CTA: orders none of
+// this thread's earlier memory operations. Use it only where the caller has
+// made the arrive wait for what it guards by other means (a store that
+// consumes every value it loaded, issued before the arrive).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_bar_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   cluster_bar_addr)
+               : "memory");
+}
+
 // Arrive (release at cluster scope) on an mbarrier that may live in the peer CTA.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
