@@ -137,6 +137,35 @@ def test_topk_heavy_ties_fallback(libs):
         assert np.array_equal(idx.cpu().numpy(), ref), k
 
 
+def test_topk_long_rows(libs):
+    """Rows of up to 70,000 scores, bit for bit against the oracle's selection:
+    random rows, a row whose large scores sit in regularly spaced 32-score runs,
+    ties around the k-th score, all-equal rows (signed zeros included),
+    non-finite values, and lengths of 16,384 and 16,389."""
+    dsa, T = libs
+    rng = np.random.default_rng(7)
+    n = 70000
+    R = 8
+    s = rng.standard_normal((R, n)).astype(np.float32)
+    n_lines = (n + 31) // 32                           # row 1: large values in spaced runs
+    for li in [q * n_lines // 256 for q in range(136)]:
+        s[1, 32 * li:32 * li + 32] = 10.0 + rng.random(32, dtype=np.float32)
+    s[2] = rng.choice(np.array([0.5, 1.0, 1.5, 3.0], dtype=np.float32), size=n,
+                      p=[0.5, 0.3, 0.17, 0.03])         # ties around the k-th score
+    s[3] = 4.0                                          # all equal
+    s[4, rng.integers(0, n, 5000)] = np.nan
+    s[4, rng.integers(0, n, 5000)] = -np.inf
+    s[4, rng.integers(0, n, 300)] = np.inf
+    s[5] = np.abs(s[5]) * np.where(rng.random(n) < 0.5, -0.0, 0.0).astype(np.float32)
+    pos = np.array([n - 1, n - 1, n - 1, 60000, n - 1, n - 1, 16383, 16388], dtype=np.int32)
+    for k in (2048, 64, 1):
+        idx = torch.empty(R, k, dtype=torch.int32, device="cuda")
+        dsa.dsa_topk(torch.from_numpy(s).cuda(), torch.from_numpy(pos).cuda(), k, idx)
+        assert dsa.dsa_check_status() == 0
+        ref = T.topk_oracle_on(s.astype(np.float64), pos, k)
+        assert np.array_equal(idx.cpu().numpy(), ref), k
+
+
 def _attention_case(dsa, T, L, k, seed, rows=None):
     inp = make_prefill(_wl(L, k), device="cuda", seed=seed)
     rng = np.random.default_rng(seed)
