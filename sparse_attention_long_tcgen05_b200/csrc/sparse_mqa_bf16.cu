@@ -64,6 +64,7 @@ constexpr int kRopeStages = 2;       // ring of CTA1's rope chunk
 constexpr int kChunkKV = kBK * 128;  // one 64-dim chunk of a key block: 64 rows x 128 B
 constexpr int kMaxK = 2048;
 constexpr int kMaxBlocks = kMaxK / kBK;
+static_assert(kMaxBlocks <= 32, "one lane of a warp per key block in the plan's compaction");
 // Warp roles. One TMA tile::gather4 request moves four 128-byte row pieces
 // and keeps its issuing warp busy ~90 cycles; measured on B200, the gather
 // rate grows with the number of issuing warps (not lanes), so 19 warps issue.
@@ -232,6 +233,19 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
   }
   const int nb = (a.k + kBK - 1) / kBK;
 
+  // The planning warps issue their index-row loads first, so the loads
+  // overlap the barrier set-up and the cluster sync below.
+  int e_in[4] = {-1, -1, -1, -1};
+  if (warp < kPlanWarps) {
+    const int32_t* irow = a.idx + static_cast<int64_t>(qi) * a.ld_idx;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int b = 2 * warp + (i >> 1);
+      const int jj = b * kBK + (i & 1) * 32 + lane;
+      if (b < nb && jj < a.k) e_in[i] = __ldg(irow + jj);
+    }
+  }
+
   if (threadIdx.x == 0) {
     mbar_init(&S.plan_full, 1);
     mbar_init(&S.q_full, 3 * 128);
@@ -268,16 +282,13 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
     regs_dec<kRegsSmall>();
     if (warp < kPlanWarps) {
       // ---------------------------------------------------------- plan (warps 0-15)
-      const int32_t* irow = a.idx + static_cast<int64_t>(qi) * a.ld_idx;
       // warp w scans blocks 2w and 2w+1; e[2i + half] holds entry
       // (2w + i) * 64 + 32 half + lane
       int e[4];
       bool bad = false;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int b = 2 * warp + (i >> 1);
-        const int jj = b * kBK + (i & 1) * 32 + lane;
-        e[i] = (b < nb && jj < a.k) ? __ldg(irow + jj) : -1;
+        e[i] = e_in[i];
         bad |= e[i] > pos;
         e[i] = (e[i] >= 0 && e[i] <= pos) ? e[i] : -1;
       }
@@ -315,19 +326,21 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
       if (rank == 0 && __any_sync(0xffffffffu, bad) && lane == 0)
         report(a.status, DSA_ERR_DEVICE_BOUNDS);
       named_bar_sync(1, kPlanWarps * 32);
-      if (threadIdx.x == 0) {
-        int nvb = 0;
-        for (int b = 0; b < nb; ++b) {
-          const uint32_t m0 = S.bmask[b][0], m1 = S.bmask[b][1];
-          if ((m0 | m1) != 0u) {
-            S.mask[nvb][0] = m0;
-            S.mask[nvb][1] = m1;
-            S.blk[nvb] = b;
-            ++nvb;
-          }
+      if (warp == 0) {
+        // compaction of the non-empty blocks: lane b looks at block b
+        const uint32_t m0 = lane < nb ? S.bmask[lane][0] : 0u;
+        const uint32_t m1 = lane < nb ? S.bmask[lane][1] : 0u;
+        const bool live = (m0 | m1) != 0u;
+        const uint32_t bal = __ballot_sync(0xffffffffu, live);
+        if (live) {
+          const int slot = __popc(bal & ((1u << lane) - 1u));
+          S.mask[slot][0] = m0;
+          S.mask[slot][1] = m1;
+          S.blk[slot] = lane;
         }
-        S.n_blocks = nvb;
-        mbar_arrive(&S.plan_full);
+        if (lane == 0) S.n_blocks = __popc(bal);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.plan_full);
       }
     }
     if (warp != kMmaWarp) {
