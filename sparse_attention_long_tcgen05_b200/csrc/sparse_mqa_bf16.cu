@@ -11,7 +11,8 @@
 //
 // B200 design. The fp32 output of 128 heads x 512 values would fill all 512
 // TMEM columns of one SM, so one query runs on a CLUSTER OF TWO CTAs that split
-// the 576 key dimensions: CTA0 owns dims [0,256), CTA1 owns [256,576). Each CTA
+// the 576 key dimensions: CTA0 owns dims [0,256), CTA1 [256,512), and the 64 rope
+// dims are split by key (see below). Each CTA
 //   - keeps its slice of Q in TMEM (the MMA's A operand read from tensor
 //     memory) and gathers only its column range of the selected rows with TMA
 //     tile::gather4 (four 128-byte row pieces per request, 128B-swizzled on
@@ -49,8 +50,11 @@
 //   warps 24-27  send the peer's partial S (lanes 32s+16 .. 32s+31);
 //   warps 28-31  take in the peer's P rows and rescale factors, rescale the
 //                peer's O rows here, and write those rows at the end.
-// CTA1's 64 rope dims are needed only by QK^T, so they sit in a ring of their
-// own that is released as soon as QK^T has read them.
+// The 64 rope dims are needed only by QK^T. Each CTA gathers them for its own
+// 32 keys of a block (CTA r: keys 32r .. 32r+31) into a ring of their own,
+// released as soon as QK^T has read it, and adds their term to those 32
+// columns of its partial S; with 4 value chunks plus half a rope chunk each,
+// the pair issues 72 gather requests per CTA and block.
 #include "dsa_common.cuh"
 #include "dsa_kernels.h"
 
@@ -60,7 +64,7 @@ namespace {
 constexpr int kH = 128;              // query heads = MMA M
 constexpr int kBK = 64;              // keys per block = QK^T MMA N
 constexpr int kStages = 4;           // ring of the four 64-dim value chunks of a key block
-constexpr int kRopeStages = 2;       // ring of CTA1's rope chunk
+constexpr int kRopeStages = 2;       // ring of the rope chunk of this CTA's 32 keys
 constexpr int kChunkKV = kBK * 128;  // one 64-dim chunk of a key block: 64 rows x 128 B
 constexpr int kMaxK = 2048;
 constexpr int kMaxBlocks = kMaxK / kBK;
@@ -92,7 +96,7 @@ constexpr uint32_t kRxPBytes = 64 * 128 + 64 * 4;   // the peer's 64 P rows + re
 
 struct __align__(1024) Smem {
   uint8_t kv[kStages][4][kChunkKV];           // 128 KB value-chunk ring
-  uint8_t rope[kRopeStages][kChunkKV];        // 16 KB rope-chunk ring (CTA1)
+  uint8_t rope[kRopeStages][kChunkKV / 2];    // 8 KB: rope dims of this CTA's 32 keys
   uint8_t p[2][kH * 128];                     // 2 x 16 KB: P [128 rows x 64 keys] bf16
   float rx_s[64 * kBK];                       // 16 KB: the peer's partial S of our heads
   float tx_s[64 * kBK];                       // 16 KB: our partial S of the peer's heads
@@ -181,20 +185,22 @@ __device__ __forceinline__ void rescale_o_rows(uint32_t t_lane, float alpha) {
   tmem_wait_st();
 }
 
-// Stages 64-dim chunks cs[] (those below nch) of this thread's Q row into
-// TMEM columns 32 c of taddr_q, all loads issued before the first store.
+// Stages 64-dim Q chunks cs[] of this thread's Q row into TMEM columns 32 c of
+// taddr_q: chunk c < 4 is dims col0 + 64c .., chunk 4 the rope dims 512 ..;
+// all loads are issued before the first store.
 template <int N>
-__device__ __forceinline__ void stage_q_chunks(uint32_t taddr_q, const uint4* src,
-                                               const int (&cs)[N], int nch) {
+__device__ __forceinline__ void stage_q_chunks(uint32_t taddr_q, const uint4* qrow, int col0,
+                                               const int (&cs)[N]) {
   uint4 qv[8 * N];
 #pragma unroll
-  for (int k = 0; k < N; ++k)
+  for (int k = 0; k < N; ++k) {
+    const uint4* src = qrow + (cs[k] < 4 ? col0 + 64 * cs[k] : 512) / 8;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      qv[8 * k + i] = cs[k] < nch ? __ldg(src + cs[k] * 8 + i) : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < 8; ++i) qv[8 * k + i] = __ldg(src + i);
+  }
 #pragma unroll
   for (int k = 0; k < N; ++k) {
-    if (cs[k] < nch) {
+    {
       uint32_t w[32];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -218,7 +224,6 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();     // 0 or 1
   const uint32_t peer = rank ^ 1u;
-  const int nch = 4 + static_cast<int>(rank);  // 64-dim chunks owned by this CTA
   const int col0 = 256 * static_cast<int>(rank);
   const int qi = blockIdx.x >> 1;
 
@@ -345,10 +350,10 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
     }
     if (warp != kMmaWarp) {
       // ---------------------------------------------------------- gather (19 issuing warps)
-      // Block j's 16 groups of 4 rows x nch 64-dim chunks are split over the
-      // issuers: issuer i requests pieces p = i, i + 19, ... (group p / nch,
-      // chunk p % nch), each landing as 4 swizzled 128-byte rows; chunk 4
-      // (CTA1's rope dims) goes to the rope ring.
+      // Block j's 16 groups of 4 rows x 4 64-dim value chunks, plus the rope
+      // chunk of this CTA's 8 groups (keys 32 rank ..), are split over the
+      // issuers: issuer i requests pieces p = i, i + 19, ...; each lands as 4
+      // swizzled 128-byte rows.
       // Only issuer 0 waits on the ring's barriers; the other 18 warps sleep on
       // hardware named barrier 2 (taking no issue slots from the softmax warps)
       // and learn from a shared flag whether to go on, so all 19 always take
@@ -360,20 +365,20 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
       }
       named_bar_sync(2, kGatherIssuers * 32);
       const int n = S.gather_n;
-      const int n_req = (kBK / 4) * nch;
+      const int n_req = (kBK / 4) * 4 + kBK / 8;
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
         const int rs = j % kRopeStages;
         if (issuer == 0) {
           bool ok = mbar_wait_warp(&S.kv_empty[st], static_cast<uint32_t>((j / kStages) & 1) ^ 1u,
                                    a.status);
-          if (ok && rank == 1)
+          if (ok)
             ok = mbar_wait_warp(&S.rope_empty[rs],
                                 static_cast<uint32_t>((j / kRopeStages) & 1) ^ 1u, a.status);
           if (lane == 0) {
             if (ok) {
               mbar_arrive_expect_tx(&S.kv_full[st], 4 * kChunkKV);
-              if (rank == 1) mbar_arrive_expect_tx(&S.rope_full[rs], kChunkKV);
+              mbar_arrive_expect_tx(&S.rope_full[rs], kChunkKV / 2);
             }
             S.gather_go[j & 1] = ok ? 1 : 0;
           }
@@ -383,14 +388,17 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
         if (lane == 0) {
           const int* rb = S.rows + S.blk[j] * kBK;
           for (int p = issuer; p < n_req; p += kGatherIssuers) {
-            const int g = p / nch, c = p - g * nch;
-            const int4 r4 = *reinterpret_cast<const int4*>(rb + 4 * g);
-            if (c < 4)
+            if (p < (kBK / 4) * 4) {
+              const int g = p >> 2, c = p & 3;
+              const int4 r4 = *reinterpret_cast<const int4*>(rb + 4 * g);
               tma_gather4(S.kv[st][c] + g * 512, &a.map_kv, col0 + 64 * c, r4.x, r4.y, r4.z,
                           r4.w, &S.kv_full[st]);
-            else
-              tma_gather4(S.rope[rs] + g * 512, &a.map_kv, 512, r4.x, r4.y, r4.z, r4.w,
+            } else {
+              const int gg = p - (kBK / 4) * 4;                  // 0..7
+              const int4 r4 = *reinterpret_cast<const int4*>(rb + 4 * (8 * rank + gg));
+              tma_gather4(S.rope[rs] + gg * 512, &a.map_kv, 512, r4.x, r4.y, r4.z, r4.w,
                           &S.rope_full[rs]);
+            }
           }
         }
         __syncwarp();
@@ -398,6 +406,7 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
     } else {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc_qk = make_idesc(kBK, 1, 1, 0, 0);   // bf16, A (TMEM) and B K-major
+      const uint32_t idesc_rope = make_idesc(kBK / 2, 1, 1, 0, 0);   // this CTA's 32 keys
       const uint32_t idesc_pv = make_idesc(256, 1, 1, 0, 1);   // bf16, K-major P, MN-major V
       bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
       const int n = ok ? S.n_blocks : 0;
@@ -410,8 +419,7 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
         if (!mbar_wait_warp(&S.kv_full[st], static_cast<uint32_t>(jj / kStages) & 1u,
                             a.status))
           return false;
-        if (rank == 1 &&
-            !mbar_wait_warp(&S.rope_full[rs], static_cast<uint32_t>(jj / kRopeStages) & 1u,
+        if (!mbar_wait_warp(&S.rope_full[rs], static_cast<uint32_t>(jj / kRopeStages) & 1u,
                             a.status))
           return false;
         if (!mbar_wait_warp(&S.s_empty, static_cast<uint32_t>((jj & 1) ^ 1), a.status))
@@ -419,16 +427,21 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
         tc_fence_after();
         if (lane == 0) {
           const uint32_t d = tmem_base + kColS;
-          for (int c = 0; c < nch; ++c) {
-            const uint64_t kd =
-                sw128_desc(smem_u32(c < 4 ? S.kv[st][c] : S.rope[rs]), 16, 1024);
+          for (int c = 0; c < 4; ++c) {
+            const uint64_t kd = sw128_desc(smem_u32(S.kv[st][c]), 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_bf16_ts(d, tmem_base + kColQ + c * 32 + kk * 8, kd + 2 * kk, idesc_qk,
                           (c | kk) != 0 ? 1u : 0u);
           }
+          // rope term of this CTA's 32 keys, into their S columns
+          const uint64_t rd = sw128_desc(smem_u32(S.rope[rs]), 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(d + 32u * rank, tmem_base + kColQ + 4 * 32 + kk * 8, rd + 2 * kk,
+                        idesc_rope, 1u);
           mma_commit(&S.s_full);
-          if (rank == 1) mma_commit(&S.rope_empty[rs]);
+          mma_commit(&S.rope_empty[rs]);
         }
         __syncwarp();
         return true;
@@ -472,14 +485,13 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
     const uint32_t lane_q = static_cast<uint32_t>(32 * s) << 16;
     // Q -> TMEM (32x32b: thread = lane 32s + lane). Row order: lane 32s+i is
     // own head 64 rank + 16s + i, lane 32s+16+i the peer's head.
-    const uint4* qsrc = reinterpret_cast<const uint4*>(
+    const uint4* qrow = reinterpret_cast<const uint4*>(
         a.q + static_cast<int64_t>(qi) * a.ld_q +
         static_cast<int64_t>(64 * static_cast<int>(rank ^ static_cast<uint32_t>(lane >> 4)) +
-                             16 * s + (lane & 15)) * 576 +
-        col0);
+                             16 * s + (lane & 15)) * 576);
     {
       const int cs[3] = {0, 3, 4};   // the send and receive warps stage 1 and 2
-      stage_q_chunks(tmem_base + lane_q + kColQ, qsrc, cs, nch);
+      stage_q_chunks(tmem_base + lane_q + kColQ, qrow, col0, cs);
       tc_fence_before();
       mbar_arrive(&S.q_full);
     }
@@ -624,14 +636,13 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
     const uint32_t lane_q = static_cast<uint32_t>(32 * s) << 16;
     // Q -> TMEM (32x32b: thread = lane 32s + lane). Row order: lane 32s+i is
     // own head 64 rank + 16s + i, lane 32s+16+i the peer's head.
-    const uint4* qsrc = reinterpret_cast<const uint4*>(
+    const uint4* qrow = reinterpret_cast<const uint4*>(
         a.q + static_cast<int64_t>(qi) * a.ld_q +
         static_cast<int64_t>(64 * static_cast<int>(rank ^ static_cast<uint32_t>(lane >> 4)) +
-                             16 * s + (lane & 15)) * 576 +
-        col0);
+                             16 * s + (lane & 15)) * 576);
     {
       const int cs[1] = {warp < kRecvWarp0 ? 1 : 2};
-      stage_q_chunks(tmem_base + lane_q + kColQ, qsrc, cs, nch);
+      stage_q_chunks(tmem_base + lane_q + kColQ, qrow, col0, cs);
       tc_fence_before();
       mbar_arrive(&S.q_full);
     }
