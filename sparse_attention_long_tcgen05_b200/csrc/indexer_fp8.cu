@@ -23,7 +23,11 @@
 //   warp 1    TMEM owner and single-thread MMA issuer (2 accumulators in TMEM)
 //   warps 2-9 epilogue, two warps per TMEM sub-partition: warps 2-5 reduce
 //             queries 0-1 of the group, warps 6-9 queries 2-3;
-//             tcgen05.ld -> ReLU * w -> head sum -> * sk -> global
+//             tcgen05.ld -> ReLU * w -> head sum -> * sk -> global.
+//             With one query per group (paged decode) each MMA step covers
+//             two key tiles, one per 64-column half of a 128-column
+//             accumulator, and warps 2-5 reduce the first, warps 6-9 the
+//             second, so both halves of the epilogue work.
 // A work unit is (group of G query rows, run of up to 16 key tiles of 128).
 #include "dsa_common.cuh"
 #include "dsa_kernels.h"
@@ -137,9 +141,9 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&S.k_full[i], 1);
-      // released by the MMAs' completion and by every epilogue thread once it
-      // has read the stage's key scales
-      mbar_init(&S.k_empty[i], 1 + kEpiThreads);
+      // released by the MMAs' completion and by every epilogue thread that
+      // reads the stage's key scales (half of them with one query per group)
+      mbar_init(&S.k_empty[i], 1 + (G == 1 ? kEpiThreads / 2 : kEpiThreads));
     }
     fence_barrier_init();
   }
@@ -156,35 +160,46 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int it = 0, ks = 0;
-      uint32_t kph = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-        const Unit U = get_unit(a, G, n_chunks, n_tiles, u, true);
-        const int qb = it & 1;
-        const uint32_t qph = (it >> 1) & 1;
-        if (!mbar_wait(&S.q_empty[qb], qph ^ 1, a.status)) { ok = false; break; }
+    // Lane 0 issues the TMA loads; in paged mode the whole warp first reads the
+    // unit's (at most 32) block-table entries in one coalesced load, so no key
+    // tile waits on a dependent page lookup.
+    int it = 0, ks = 0;
+    uint32_t kph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
+      const Unit U = get_unit(a, G, n_chunks, n_tiles, u, lane == 0);
+      const int qb = it & 1;
+      const uint32_t qph = (it >> 1) & 1;
+      if (!mbar_wait_warp(&S.q_empty[qb], qph ^ 1, a.status)) { ok = false; break; }
+      if (lane == 0) {
         mbar_arrive_expect_tx(&S.q_full[qb], U.ng * kQBytes);
         for (int i = 0; i < U.ng; ++i)
           tma_load_3d(S.q[qb] + i * kQBytes, &a.map_q, 0, 0, U.qi[i], &S.q_full[qb]);
-        for (int t = U.t0; t < U.t_end; ++t) {
-          if (!mbar_wait(&S.k_empty[ks], kph ^ 1, a.status)) { ok = false; break; }
+      }
+      int pg = -1;     // page of logical page 2 t0 + lane, if it holds a key <= max_pos
+      if (a.keys.paged) {
+        const int p = 2 * U.t0 + lane;
+        if (lane < 2 * (U.t_end - U.t0) && p * 64 <= U.max_pos) pg = page_of(a, U.qi[0], p, true);
+      }
+      for (int t = U.t0; t < U.t_end; ++t) {
+        if (!mbar_wait_warp(&S.k_empty[ks], kph ^ 1, a.status)) { ok = false; break; }
+        const int i0 = 2 * (t - U.t0);
+        const int pg0 = __shfl_sync(0xffffffffu, pg, i0 & 31);
+        const int pg1 = __shfl_sync(0xffffffffu, pg, (i0 + 1) & 31);
+        if (lane == 0) {
           mbar_arrive_expect_tx(&S.k_full[ks], kKBytes + kSkBytes);
           if (!a.keys.paged) {
             tma_load_2d(S.k[ks], &a.map_k, 0, t * kKeyTile, &S.k_full[ks]);
             tma_load_1d(S.sk[ks], &a.map_sk, t * kKeyTile, &S.k_full[ks]);
           } else {
-            const int p0 = 2 * t;
-            const int pg0 = page_of(a, U.qi[0], p0, true);
-            const int pg1 = (p0 + 1) * 64 <= U.max_pos ? page_of(a, U.qi[0], p0 + 1, true) : pg0;
+            const int pg1u = pg1 >= 0 ? pg1 : pg0;   // second page past max_pos: reuse the first
             tma_load_2d(S.k[ks], &a.map_k, 0, pg0 * 64, &S.k_full[ks]);
-            tma_load_2d(S.k[ks] + kKBytes / 2, &a.map_k, 0, pg1 * 64, &S.k_full[ks]);
+            tma_load_2d(S.k[ks] + kKBytes / 2, &a.map_k, 0, pg1u * 64, &S.k_full[ks]);
             tma_load_1d(S.sk[ks], &a.map_sk, pg0 * 64, &S.k_full[ks]);
-            tma_load_1d(S.sk[ks] + 64, &a.map_sk, pg1 * 64, &S.k_full[ks]);
+            tma_load_1d(S.sk[ks] + 64, &a.map_sk, pg1u * 64, &S.k_full[ks]);
           }
-          if (++ks == kStages) { ks = 0; kph ^= 1; }
         }
+        if (++ks == kStages) { ks = 0; kph ^= 1; }
       }
     }
   } else if (warp == 1) {
@@ -201,6 +216,36 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
         if (!mbar_wait(&S.q_full[qb], qph, a.status)) break;
         tc_fence_after();
         const uint64_t bdesc = sw128_desc(smem_u32(S.q[qb]), 16, 1024);
+        if (G == 1) {
+          // two key tiles per step, into the two 64-column halves of a
+          // 128-column accumulator
+          for (int t = U.t0; t < U.t_end && ok; t += 2) {
+            const int nt = min(2, U.t_end - t);
+            if (!mbar_wait(&S.acc_empty[ab], aph ^ 1, a.status)) { ok = false; break; }
+            for (int h = 0; h < nt && ok; ++h) {
+              const int kss = ks + h < kStages ? ks + h : ks + h - kStages;
+              const uint32_t kp = ks + h < kStages ? kph : kph ^ 1u;
+              if (!mbar_wait(&S.k_full[kss], kp, a.status)) ok = false;
+            }
+            if (!ok) break;
+            tc_fence_after();
+            for (int h = 0; h < nt; ++h) {
+              const int kss = ks + h < kStages ? ks + h : ks + h - kStages;
+              const uint64_t adesc = sw128_desc(smem_u32(S.k[kss]), 16, 1024);
+              const uint32_t d = tmem_base + static_cast<uint32_t>(ab * 2 * N + h * N);
+#pragma unroll
+              for (int kk = 0; kk < kDim / 32; ++kk)
+                mma_f8(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+              mma_commit(&S.k_empty[kss]);
+            }
+            mma_commit(&S.acc_full[ab]);
+            for (int h = 0; h < nt; ++h)
+              if (++ks == kStages) { ks = 0; kph ^= 1; }
+            if (++ab == 2) { ab = 0; aph ^= 1; }
+          }
+          mma_commit(&S.q_empty[qb]);
+          continue;
+        }
         for (int t = U.t0; t < U.t_end; ++t) {
           if (!mbar_wait(&S.k_full[ks], kph, a.status) ||
               !mbar_wait(&S.acc_empty[ab], aph ^ 1, a.status)) { ok = false; break; }
@@ -237,6 +282,50 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
         S.wq[i] = a.w[static_cast<int64_t>(qi) * a.ld_w + (i % kHeads)] * a.q_scale[qi];
       }
       named_bar_sync(1, kEpiThreads);
+      if (G == 1) {
+        // one query; half h reduces the second key tile of each step if h = 1
+        float* const srow = a.scores + static_cast<int64_t>(U.row0) * a.ld_scores;
+        const int my_pos = U.pos[0];
+        if (a.write_masked)
+          for (int t = max(U.t0, U.t_end) + half; t < U.t1; t += 2) {
+            const int s = t * kKeyTile + sub * 32 + lane;
+            if (s < a.n_cols) srow[s] = -INFINITY;
+          }
+        for (int t = U.t0; t < U.t_end && ok; t += 2) {
+          const int nt = min(2, U.t_end - t);
+          const bool mine = half < nt;
+          const int s = (t + half) * kKeyTile + sub * 32 + lane;
+          float sk = 0.f;
+          if (mine) {
+            const int kss = ks + half < kStages ? ks + half : ks + half - kStages;
+            const uint32_t kp = ks + half < kStages ? kph : kph ^ 1u;
+            if (!mbar_wait_warp(&S.k_full[kss], kp, a.status)) { ok = false; break; }
+            sk = S.sk[kss][sub * 32 + lane];
+            mbar_arrive(&S.k_empty[kss]);
+          }
+          if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status)) { ok = false; break; }
+          tc_fence_after();
+          if (mine) {
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) +
+                                   static_cast<uint32_t>(ab * 2 * N + half * N);
+            uint32_t r0[32], r1[32];
+            tmem_ld32(tbase, r0);
+            tmem_ld32(tbase + 32, r1);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&S.acc_empty[ab]);
+            const float s0 = indexer_score_from_dots(r0, r1, &S.wq[0], sk);
+            if (s < a.n_cols) srow[s] = s <= my_pos ? s0 : -INFINITY;
+          } else {
+            tc_fence_before();
+            mbar_arrive(&S.acc_empty[ab]);
+          }
+          for (int h = 0; h < nt; ++h)
+            if (++ks == kStages) { ks = 0; kph ^= 1; }
+          if (++ab == 2) { ab = 0; aph ^= 1; }
+        }
+        continue;
+      }
       const int g0 = 2 * half;                          // first query of this warp
       const int nq = max(0, min(2, U.ng - g0));         // queries this warp reduces
       for (int t = U.t0; t < U.t1 && ok; ++t) {
