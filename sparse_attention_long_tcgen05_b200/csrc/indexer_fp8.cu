@@ -19,7 +19,10 @@
 //
 // Roles (320 threads, one CTA per SM, persistent over work units):
 //   warp 0    TMA producer: Q group (once per unit), key tiles and their fp32
-//             key scales through a 6-stage ring
+//             key scales through a 6-stage ring; in paged mode it loads the
+//             first 64-key page of each tile and warp 10 the second (a TMA
+//             load keeps its issuing warp busy for ~100 cycles, and a paged
+//             tile takes four of them)
 //   warp 1    TMEM owner and single-thread MMA issuer (2 accumulators in TMEM)
 //   warps 2-9 epilogue, two warps per TMEM sub-partition: warps 2-5 reduce
 //             queries 0-1 of the group, warps 6-9 queries 2-3;
@@ -44,7 +47,8 @@ constexpr int kStages = 6;
 constexpr int kTilesPerUnit = 16;
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kThreads = 64 + kEpiThreads;
+constexpr int kThreads = 64 + kEpiThreads + 32;   // + warp 10, second paged producer
+constexpr int kPageWarp = 2 + kEpiWarps;
 constexpr int kQBytes = kHeads * kDim;      // 8 KB per query
 constexpr int kKBytes = kKeyTile * kDim;    // 16 KB per key tile
 constexpr int kSkBytes = kKeyTile * 4;      // 512 B of key scales per tile
@@ -158,28 +162,34 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || (warp == kPageWarp && a.keys.paged)) {
+    // ------------------------------------------------------------ producer(s)
     // Lane 0 issues the TMA loads; in paged mode the whole warp first reads the
     // unit's (at most 32) block-table entries in one coalesced load, so no key
-    // tile waits on a dependent page lookup.
+    // tile waits on a dependent page lookup. Warp 0 loads the query group,
+    // arms the stage's barrier for the whole tile and loads its first page (or
+    // the whole contiguous tile); warp 10 loads the second page of a paged tile.
+    const bool first = warp == 0;
     int it = 0, ks = 0;
     uint32_t kph = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-      const Unit U = get_unit(a, G, n_chunks, n_tiles, u, lane == 0);
+      const Unit U = get_unit(a, G, n_chunks, n_tiles, u, first && lane == 0);
       const int qb = it & 1;
       const uint32_t qph = (it >> 1) & 1;
-      if (!mbar_wait_warp(&S.q_empty[qb], qph ^ 1, a.status)) { ok = false; break; }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&S.q_full[qb], U.ng * kQBytes);
-        for (int i = 0; i < U.ng; ++i)
-          tma_load_3d(S.q[qb] + i * kQBytes, &a.map_q, 0, 0, U.qi[i], &S.q_full[qb]);
+      if (first) {
+        if (!mbar_wait_warp(&S.q_empty[qb], qph ^ 1, a.status)) { ok = false; break; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&S.q_full[qb], U.ng * kQBytes);
+          for (int i = 0; i < U.ng; ++i)
+            tma_load_3d(S.q[qb] + i * kQBytes, &a.map_q, 0, 0, U.qi[i], &S.q_full[qb]);
+        }
       }
       int pg = -1;     // page of logical page 2 t0 + lane, if it holds a key <= max_pos
       if (a.keys.paged) {
         const int p = 2 * U.t0 + lane;
-        if (lane < 2 * (U.t_end - U.t0) && p * 64 <= U.max_pos) pg = page_of(a, U.qi[0], p, true);
+        if (lane < 2 * (U.t_end - U.t0) && p * 64 <= U.max_pos)
+          pg = page_of(a, U.qi[0], p, first);
       }
       for (int t = U.t0; t < U.t_end; ++t) {
         if (!mbar_wait_warp(&S.k_empty[ks], kph ^ 1, a.status)) { ok = false; break; }
@@ -187,15 +197,16 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
         const int pg0 = __shfl_sync(0xffffffffu, pg, i0 & 31);
         const int pg1 = __shfl_sync(0xffffffffu, pg, (i0 + 1) & 31);
         if (lane == 0) {
-          mbar_arrive_expect_tx(&S.k_full[ks], kKBytes + kSkBytes);
+          if (first) mbar_arrive_expect_tx(&S.k_full[ks], kKBytes + kSkBytes);
           if (!a.keys.paged) {
             tma_load_2d(S.k[ks], &a.map_k, 0, t * kKeyTile, &S.k_full[ks]);
             tma_load_1d(S.sk[ks], &a.map_sk, t * kKeyTile, &S.k_full[ks]);
+          } else if (first) {
+            tma_load_2d(S.k[ks], &a.map_k, 0, pg0 * 64, &S.k_full[ks]);
+            tma_load_1d(S.sk[ks], &a.map_sk, pg0 * 64, &S.k_full[ks]);
           } else {
             const int pg1u = pg1 >= 0 ? pg1 : pg0;   // second page past max_pos: reuse the first
-            tma_load_2d(S.k[ks], &a.map_k, 0, pg0 * 64, &S.k_full[ks]);
             tma_load_2d(S.k[ks] + kKBytes / 2, &a.map_k, 0, pg1u * 64, &S.k_full[ks]);
-            tma_load_1d(S.sk[ks], &a.map_sk, pg0 * 64, &S.k_full[ks]);
             tma_load_1d(S.sk[ks] + 64, &a.map_sk, pg1u * 64, &S.k_full[ks]);
           }
         }
@@ -263,7 +274,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
         mma_commit(&S.q_empty[qb]);
       }
     }
-  } else {
+  } else if (warp >= 2 && warp < kPageWarp) {
     // ------------------------------------------------------------ epilogue
     const int sub = warp & 3;              // TMEM sub-partition of this warp
     const int half = (warp - 2) >> 2;      // 0: queries 0-1, 1: queries 2-3
