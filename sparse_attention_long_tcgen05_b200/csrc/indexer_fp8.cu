@@ -339,12 +339,18 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
       }
       const int g0 = 2 * half;                          // first query of this warp
       const int nq = max(0, min(2, U.ng - g0));         // queries this warp reduces
+      // this warp's two rows, selected with constant indices so U stays in registers
+      const int pos0 = half ? U.pos[2] : U.pos[0];
+      const int pos1 = half ? U.pos[3] : U.pos[1];
+      float* const srow0 = a.scores + static_cast<int64_t>(U.row0 + g0) * a.ld_scores;
+      float* const srow1 = srow0 + a.ld_scores;
       for (int t = U.t0; t < U.t1 && ok; ++t) {
         const int s = t * kKeyTile + sub * 32 + lane;
         if (t >= U.t_end) {
-          if (a.write_masked && s < a.n_cols)
-            for (int gq = 0; gq < nq; ++gq)
-              a.scores[static_cast<int64_t>(U.row0 + g0 + gq) * a.ld_scores + s] = -INFINITY;
+          if (a.write_masked && s < a.n_cols) {
+            if (nq > 0) srow0[s] = -INFINITY;
+            if (nq > 1) srow1[s] = -INFINITY;
+          }
           continue;
         }
         // this tile's key scale (the stage also holds the key codes)
@@ -368,10 +374,8 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           const float s0 = indexer_score_from_dots(r0, r1, &S.wq[g0 * kHeads], sk);
           const float s1 = indexer_score_from_dots(r2, r3, &S.wq[(g0 + 1) * kHeads], sk);
           if (s < a.n_cols) {
-            a.scores[static_cast<int64_t>(U.row0 + g0) * a.ld_scores + s] =
-                s <= U.pos[g0] ? s0 : -INFINITY;
-            a.scores[static_cast<int64_t>(U.row0 + g0 + 1) * a.ld_scores + s] =
-                s <= U.pos[g0 + 1] ? s1 : -INFINITY;
+            srow0[s] = s <= pos0 ? s0 : -INFINITY;
+            srow1[s] = s <= pos1 ? s1 : -INFINITY;
           }
         } else if (nq == 1) {
           uint32_t r0[32], r1[32];
@@ -381,9 +385,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           tc_fence_before();
           mbar_arrive(&S.acc_empty[ab]);
           const float s0 = indexer_score_from_dots(r0, r1, &S.wq[g0 * kHeads], sk);
-          if (s < a.n_cols)
-            a.scores[static_cast<int64_t>(U.row0 + g0) * a.ld_scores + s] =
-                s <= U.pos[g0] ? s0 : -INFINITY;
+          if (s < a.n_cols) srow0[s] = s <= pos0 ? s0 : -INFINITY;
         } else {
           tc_fence_before();
           mbar_arrive(&S.acc_empty[ab]);

@@ -8,7 +8,8 @@
 // order, padded with -1 when t+1 < k.
 //
 // One CTA (1024 threads) per row, scores compared as order-preserving uint32
-// keys. Two passes over the row:
+// keys, rows read as float4 where their alignment allows. Two passes over the
+// row:
 //   1. a histogram of the top 12 key bits finds the bin b1 holding the k-th
 //      largest key;
 //   2. an ordered collection (warp ballots, one block scan per 8192 scores)
@@ -231,9 +232,35 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
     return;
   }
 
+  // Rows that start on a 16-byte boundary with a row pitch of whole float4s
+  // are read as float4: the float4 holding the last score stays inside the
+  // row, and a lane keeps four loads in flight where it had one.
+  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15u) == 0 && (a.ld_scores & 3) == 0;
+  const float4* row4 = reinterpret_cast<const float4*>(row);
+
   // ---- pass 1: histogram of the top 12 key bits
   clear_hist(S.hist, 4096);
-  for (int i = tid; i < n; i += kThreads) atomicAdd(&S.hist[order_key(row[i]) >> 20], 1u);
+  if (vec) {
+    const int n4 = (n + 3) >> 2;
+    for (int c = tid; c < n4; c += 4 * kThreads) {
+      float4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int q = c + j * kThreads;
+        v[j] = q < n4 ? row4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = 4 * (c + j * kThreads);
+        if (i < n) atomicAdd(&S.hist[order_key(v[j].x) >> 20], 1u);
+        if (i + 1 < n) atomicAdd(&S.hist[order_key(v[j].y) >> 20], 1u);
+        if (i + 2 < n) atomicAdd(&S.hist[order_key(v[j].z) >> 20], 1u);
+        if (i + 3 < n) atomicAdd(&S.hist[order_key(v[j].w) >> 20], 1u);
+      }
+    }
+  } else {
+    for (int i = tid; i < n; i += kThreads) atomicAdd(&S.hist[order_key(row[i]) >> 20], 1u);
+  }
   __syncthreads();
   find_bin(S.hist, 4096, static_cast<uint32_t>(k), S.warp_sums, S.found);
   const uint32_t b1 = S.found[0];
@@ -244,29 +271,68 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
     return;
   }
 
-  // ---- pass 2: collect keys in bins >= b1 with their indices, in index order
+  // ---- pass 2: collect keys in bins >= b1 with their indices, in index order.
+  // Warp w takes scores [c0 + 256 w, c0 + 256 w + 256) of a chunk: two slices
+  // of 128, lane l holding scores 4l..4l+3 of a slice (float4 rows) or, for
+  // other rows, scores j*32 + l.
   const uint32_t lt = (1u << lane) - 1u;
   uint32_t base = 0;
   for (int c0 = 0; c0 < n; c0 += kChunk) {
     uint32_t bal[kPer], key[kPer];
     uint32_t cnt = 0;
+    const int wbase = c0 + w * (32 * kPer);
+    if (vec) {
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int i = c0 + w * (32 * kPer) + j * 32 + lane;
-      key[j] = i < n ? order_key(row[i]) : 0u;
-      bal[j] = __ballot_sync(0xffffffffu, i < n && (key[j] >> 20) >= b1);
-      cnt += __popc(bal[j]);
+      for (int h = 0; h < kPer / 4; ++h) {
+        const int i0 = wbase + h * 128 + 4 * lane;
+        const float4 v = i0 < n ? row4[i0 >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+        key[4 * h + 0] = i0 < n ? order_key(v.x) : 0u;
+        key[4 * h + 1] = i0 + 1 < n ? order_key(v.y) : 0u;
+        key[4 * h + 2] = i0 + 2 < n ? order_key(v.z) : 0u;
+        key[4 * h + 3] = i0 + 3 < n ? order_key(v.w) : 0u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          bal[4 * h + e] = __ballot_sync(0xffffffffu, i0 + e < n && (key[4 * h + e] >> 20) >= b1);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = wbase + j * 32 + lane;
+        key[j] = i < n ? order_key(row[i]) : 0u;
+        bal[j] = __ballot_sync(0xffffffffu, i < n && (key[j] >> 20) >= b1);
+      }
     }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) cnt += __popc(bal[j]);
     uint32_t total;
     uint32_t off = base + warp_excl_scan(cnt, S.warp_sums, total);
+    if (vec) {
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      if ((bal[j] >> lane) & 1u) {
-        const uint32_t p = off + __popc(bal[j] & lt);
-        S.lidx[p] = c0 + w * (32 * kPer) + j * 32 + lane;
-        S.lkey[p] = key[j];
+      for (int h = 0; h < kPer / 4; ++h) {
+        uint32_t p = off;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) p += __popc(bal[4 * h + e] & lt);
+        const int i0 = wbase + h * 128 + 4 * lane;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if ((bal[4 * h + e] >> lane) & 1u) {
+            S.lidx[p] = i0 + e;
+            S.lkey[p] = key[4 * h + e];
+            ++p;
+          }
+          off += __popc(bal[4 * h + e]);
+        }
       }
-      off += __popc(bal[j]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        if ((bal[j] >> lane) & 1u) {
+          const uint32_t p = off + __popc(bal[j] & lt);
+          S.lidx[p] = wbase + j * 32 + lane;
+          S.lkey[p] = key[j];
+        }
+        off += __popc(bal[j]);
+      }
     }
     base += total;
   }

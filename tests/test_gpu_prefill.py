@@ -137,6 +137,27 @@ def test_topk_heavy_ties_fallback(libs):
         assert np.array_equal(idx.cpu().numpy(), ref), k
 
 
+def test_topk_row_layouts(libs):
+    """Score rows read as float4 (16-byte aligned rows, pitch a multiple of 4)
+    and rows read one score at a time (odd pitch or an unaligned first row),
+    each with ragged lengths, give the oracle's selection bit for bit."""
+    dsa, T = libs
+    rng = np.random.default_rng(11)
+    R, n = 24, 9000
+    pos = rng.integers(2040, n, R).astype(np.int32)
+    pos[:4] = [n - 1, n - 2, n - 3, n - 4]
+    for pitch, offset in ((9000, 0), (9004, 0), (9003, 0), (9004, 1), (9001, 3)):
+        buf = torch.from_numpy(rng.standard_normal(R * pitch + offset).astype(np.float32))
+        buf[offset:].view(R, pitch)[:, :n:7] = 2.5          # ties around the k-th score
+        s = buf.cuda()[offset:offset + R * pitch].view(R, pitch)[:, :n]
+        for k in (2048, 33):
+            idx = torch.empty(R, k, dtype=torch.int32, device="cuda")
+            dsa.dsa_topk(s, torch.from_numpy(pos).cuda(), k, idx)
+            assert dsa.dsa_check_status() == 0
+            ref = T.topk_oracle_on(s.double().cpu().numpy(), pos, k)
+            assert np.array_equal(idx.cpu().numpy(), ref), (pitch, offset, k)
+
+
 def test_topk_long_rows(libs):
     """Rows of up to 70,000 scores, bit for bit against the oracle's selection:
     random rows, a row whose large scores sit in regularly spaced 32-score runs,
