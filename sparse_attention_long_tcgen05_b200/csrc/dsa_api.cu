@@ -215,12 +215,19 @@ dsa_status check_attn(const dsa_attn_in* in) {
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Query rows per indexer launch inside the fused prefill: the score block of
-// one launch (rows x keys floats) stays within 64 MiB, half of the 126 MB L2.
+// Query rows per indexer launch inside the fused prefill. The score block of
+// one launch (rows x keys floats) stays resident in the 126 MB L2 between the
+// indexer that writes it and the top-k that reads it: at most 80 MiB. Its rows
+// are a multiple of 148 where that fits, so the top-k launch (one CTA per row)
+// fills the 148 SMs of a B200 in whole waves.
+constexpr int64_t kBlockFloatsMax = int64_t(20) << 20;  // 80 MiB of scores
+constexpr int64_t kRowGrain = 148;
+
 int32_t forward_chunk_rows(int32_t n_q, int32_t n_cols) {
-  int64_t c = (int64_t(16) << 20) / (n_cols > 0 ? n_cols : 1);
-  c = c < 128 ? 128 : c;
-  c = (c / 4) * 4;
+  const int64_t cols = n_cols > 0 ? n_cols : 1;
+  if (int64_t(n_q) * cols <= kBlockFloatsMax) return n_q;
+  int64_t c = kBlockFloatsMax / cols;
+  c = c >= kRowGrain ? (c / kRowGrain) * kRowGrain : (c < 128 ? 128 : (c / 4) * 4);
   return c > n_q ? n_q : static_cast<int32_t>(c);
 }
 

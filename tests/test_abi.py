@@ -47,7 +47,7 @@ def test_status_strings_and_version(lib):
 
 def test_workspace_size_host_logic(lib):
     """Workspace arithmetic needs no device: fused prefill keeps one bounded
-    block of score rows (<= 64 MiB) plus the selection."""
+    block of score rows (<= 80 MiB) plus the selection."""
     import torch
     L = 131072
     q = torch.empty(L, 64, 128, dtype=torch.uint8)
@@ -57,7 +57,7 @@ def test_workspace_size_host_logic(lib):
     ind = lib.indexer_in(q, k, w, s, s)
     nbytes = lib.dsa_workspace_size(lib.DSA_OP_FORWARD, ind, None, 0, 0, 2048)
     idx_bytes = L * 2048 * 4
-    assert idx_bytes < nbytes <= idx_bytes + (64 << 20) + 512
+    assert idx_bytes < nbytes <= idx_bytes + (80 << 20) + 512
     assert lib.dsa_workspace_size(lib.DSA_OP_SPARSE_MQA) == 0
     with pytest.raises(lib.DsaError):
         lib.dsa_workspace_size(lib.DSA_OP_FORWARD, ind, None, 0, 0, 4096)   # k > 2048

@@ -307,6 +307,22 @@ def test_forward_L4096(libs):
     _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, sample_rows(L, 64, seed=1))
 
 
+def test_forward_two_score_blocks_L5000(libs):
+    """A prefill whose scores do not fit one block (4144 rows, then a ragged
+    856): the fused selection equals the standalone top-k of the standalone
+    scores in every row."""
+    dsa, T = libs
+    inp = make_prefill(_wl(5000), device="cuda", seed=3)
+    ind, att, idx, out, lse = _forward(dsa, T, inp)
+    L, k = inp.wl.L, inp.wl.k
+    scores = torch.empty(L, L, device="cuda")
+    dsa.dsa_indexer_scores(ind, None, L, scores, L)
+    idx_s = torch.empty(L, k, dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(scores, torch.arange(L, dtype=torch.int32, device="cuda"), k, idx_s)
+    assert dsa.dsa_check_status() == 0
+    assert torch.equal(idx, idx_s)
+
+
 def test_forward_L32768_needles(libs):
     dsa, T = libs
     inp = make_prefill(WORKLOADS[2], device="cuda", seed=0)
