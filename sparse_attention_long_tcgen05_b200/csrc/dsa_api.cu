@@ -256,7 +256,7 @@ ForwardPlan forward_plan(const dsa_indexer_in& ind, int32_t k) {
 
 dsa_status run_indexer(const dsa_indexer_in& in, const int32_t* rows, int32_t q_base,
                        int32_t n_rows, float* scores, int64_t ld_scores, int32_t n_cols,
-                       int write_masked, DeviceInfo* dev, cudaStream_t stream) {
+                       int write_masked, bool pdl, DeviceInfo* dev, cudaStream_t stream) {
   const dsa::KeySide ks = key_side(in.kv, in.n_q, in.n_keys);
   if (in.dtype == DSA_E4M3) {
     dsa::IndexerFp8Args a{};
@@ -291,7 +291,7 @@ dsa_status run_indexer(const dsa_indexer_in& in, const int32_t* rows, int32_t q_
     a.n_cols = n_cols;
     a.write_masked = write_masked;
     a.status = dev->status;
-    DSA_LAUNCH(dsa::launch_indexer_fp8(a, dev->num_sms, stream));
+    DSA_LAUNCH(dsa::launch_indexer_fp8(a, dev->num_sms, pdl, stream));
     return DSA_OK;
   }
   dsa::IndexerF32Args a{};
@@ -315,7 +315,7 @@ dsa_status run_indexer(const dsa_indexer_in& in, const int32_t* rows, int32_t q_
 
 dsa_status run_topk(const float* scores, int64_t ld_scores, const int32_t* row_pos,
                     int32_t pos_minus, int32_t pos_base, int32_t n_rows, int32_t k, int32_t* idx, int64_t ld_idx,
-                    DeviceInfo* dev, cudaStream_t stream) {
+                    bool pdl, DeviceInfo* dev, cudaStream_t stream) {
   dsa::TopkArgs a{};
   a.scores = scores;
   a.ld_scores = ld_scores;
@@ -327,7 +327,7 @@ dsa_status run_topk(const float* scores, int64_t ld_scores, const int32_t* row_p
   a.idx = idx;
   a.ld_idx = ld_idx;
   a.status = dev->status;
-  DSA_LAUNCH(dsa::launch_topk(a, stream));
+  DSA_LAUNCH(dsa::launch_topk(a, pdl, stream));
   return DSA_OK;
 }
 
@@ -387,17 +387,19 @@ dsa_status run_select(const dsa_indexer_in& ind, int32_t k, int32_t* idx, int64_
                       cudaStream_t stream) {
   const int32_t n_q = ind.n_q;
   if (ind.kv.kind == DSA_KV_PAGED) {
-    DSA_TRY(run_indexer(ind, nullptr, 0, n_q, scores, p.n_cols, p.n_cols, 0, dev, stream));
+    DSA_TRY(run_indexer(ind, nullptr, 0, n_q, scores, p.n_cols, p.n_cols, 0, false, dev,
+                        stream));
     // query b sits at position ctx_lens[b] - 1
-    return run_topk(scores, p.n_cols, ind.kv.ctx_lens, 1, 0, n_q, k, idx, ld_idx, dev, stream);
+    return run_topk(scores, p.n_cols, ind.kv.ctx_lens, 1, 0, n_q, k, idx, ld_idx, true, dev,
+                    stream);
   }
   const int32_t off = ind.n_keys - n_q;  // position of query 0
   for (int32_t q0 = 0; q0 < n_q; q0 += p.chunk) {
     const int32_t rows = n_q - q0 < p.chunk ? n_q - q0 : p.chunk;
     const int32_t cols = off + q0 + rows;  // keys any query of the block sees
-    DSA_TRY(run_indexer(ind, nullptr, q0, rows, scores, cols, cols, 0, dev, stream));
+    DSA_TRY(run_indexer(ind, nullptr, q0, rows, scores, cols, cols, 0, q0 > 0, dev, stream));
     DSA_TRY(run_topk(scores, cols, nullptr, 0, off + q0, rows, k,
-                     idx + static_cast<int64_t>(q0) * ld_idx, ld_idx, dev, stream));
+                     idx + static_cast<int64_t>(q0) * ld_idx, ld_idx, true, dev, stream));
   }
   return DSA_OK;
 }
@@ -420,7 +422,7 @@ DSA_API dsa_status dsa_indexer_scores(const dsa_indexer_in* in, const int32_t* r
     return DSA_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   DSA_TRY(device_info(&dev));
-  return run_indexer(*in, rows, 0, n_rows, scores, ld_scores, n_cols, 1, dev,
+  return run_indexer(*in, rows, 0, n_rows, scores, ld_scores, n_cols, 1, false, dev,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -432,7 +434,7 @@ DSA_API dsa_status dsa_topk(const float* scores, int64_t ld_scores, const int32_
   if (k < 1 || k > kKMax || ld_idx < k) return DSA_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   DSA_TRY(device_info(&dev));
-  return run_topk(scores, ld_scores, row_pos, 0, 0, n_rows, k, idx, ld_idx, dev,
+  return run_topk(scores, ld_scores, row_pos, 0, 0, n_rows, k, idx, ld_idx, false, dev,
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -621,14 +623,17 @@ extern "C" DSA_API dsa_status dsa_select_noalloc(const dsa_indexer_in* indexer, 
     int32_t* out = idx + static_cast<int64_t>(q0) * ld_idx;
     if (paged) {
       const int32_t cols = static_cast<int32_t>(n_cols);
-      DSA_TRY(run_indexer(*indexer, nullptr, q0, rows, scratch, cols, cols, 0, dev, stream));
-      DSA_TRY(run_topk(scratch, cols, indexer->kv.ctx_lens + q0, 1, 0, rows, k, out, ld_idx, dev,
-                       stream));
+      DSA_TRY(run_indexer(*indexer, nullptr, q0, rows, scratch, cols, cols, 0, q0 > 0, dev,
+                          stream));
+      DSA_TRY(run_topk(scratch, cols, indexer->kv.ctx_lens + q0, 1, 0, rows, k, out, ld_idx,
+                       true, dev, stream));
     } else {
       const int32_t off = indexer->n_keys - n_q;
       const int32_t cols = off + q0 + rows;
-      DSA_TRY(run_indexer(*indexer, nullptr, q0, rows, scratch, cols, cols, 0, dev, stream));
-      DSA_TRY(run_topk(scratch, cols, nullptr, 0, off + q0, rows, k, out, ld_idx, dev, stream));
+      DSA_TRY(run_indexer(*indexer, nullptr, q0, rows, scratch, cols, cols, 0, q0 > 0, dev,
+                          stream));
+      DSA_TRY(run_topk(scratch, cols, nullptr, 0, off + q0, rows, k, out, ld_idx, true, dev,
+                       stream));
     }
   }
   return DSA_OK;

@@ -413,6 +413,21 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Programmatic dependent launch (PTX griddepcontrol). A kernel launched with
+// the programmatic stream serialization attribute may start while the kernel
+// before it on the stream is still running. griddep_wait() blocks the calling
+// thread until that kernel has completed and its writes are visible (it returns
+// at once for a kernel launched without the attribute); a thread must call it
+// before it touches memory that the earlier kernel reads or writes.
+// griddep_launch_dependents() lets the next kernel of the stream start early.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

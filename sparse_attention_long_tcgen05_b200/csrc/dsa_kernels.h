@@ -48,7 +48,11 @@ struct IndexerFp8Args {
   int* status;
 };
 
-cudaError_t launch_indexer_fp8(const IndexerFp8Args& a, int num_sms, cudaStream_t stream);
+// pdl: launch with programmatic stream serialization, so the kernel's set-up
+// overlaps the end of the kernel before it on the stream. Only for a launch
+// that follows another kernel of this library issued by the same call.
+cudaError_t launch_indexer_fp8(const IndexerFp8Args& a, int num_sms, bool pdl,
+                               cudaStream_t stream);
 
 struct IndexerF32Args {
   const float* q;
@@ -83,7 +87,8 @@ struct TopkArgs {
   int* status;
 };
 
-cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
+// pdl: as for launch_indexer_fp8.
+cudaError_t launch_topk(const TopkArgs& a, bool pdl, cudaStream_t stream);
 
 // ---------------------------------------------------------------- attention
 

@@ -44,7 +44,7 @@ constexpr int kDim = 128;  // e4m3 bytes per head row / per key row
 constexpr int kKeyTile = 128;
 constexpr int kMaxG = 4;
 constexpr int kStages = 6;
-constexpr int kTilesPerUnit = 16;
+constexpr int kTilesPerUnit = 16;        // largest run of key tiles in a work unit
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = 64 + kEpiThreads + 32;   // + warp 10, second paged producer
@@ -76,7 +76,7 @@ struct Unit {
 };
 
 __device__ __forceinline__ Unit get_unit(const IndexerFp8Args& a, int G, int n_chunks,
-                                         int n_tiles, int u, bool report_errors) {
+                                         int n_tiles, int tpu, int u, bool report_errors) {
   Unit U;
   const int g = u / n_chunks;
   const int c = u - g * n_chunks;
@@ -109,8 +109,8 @@ __device__ __forceinline__ Unit get_unit(const IndexerFp8Args& a, int G, int n_c
       U.max_pos = max(U.max_pos, pos);
     }
   }
-  U.t0 = c * kTilesPerUnit;
-  U.t1 = min(n_tiles, U.t0 + kTilesPerUnit);
+  U.t0 = c * tpu;
+  U.t1 = min(n_tiles, U.t0 + tpu);
   const int last = U.max_pos >= 0 ? U.max_pos / kKeyTile + 1 : 0;
   U.t_end = max(U.t0, min(U.t1, last));
   return U;
@@ -128,13 +128,17 @@ __device__ __forceinline__ int page_of(const IndexerFp8Args& a, int qi, int p, b
 
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks, int n_tiles,
-                   int n_units) {
+                   int tpu, int n_units) {
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                      ~uintptr_t(1023));
   const int warp = warp_id();
   const int lane = threadIdx.x & 31;
   const int N = G * kHeads;
+  // Only the epilogue touches memory that a kernel before this one on the
+  // stream uses (the score rows a previous top-k may still be reading); it
+  // waits for that kernel below. Everything else may start at once.
+  griddep_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -174,7 +178,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
     uint32_t kph = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-      const Unit U = get_unit(a, G, n_chunks, n_tiles, u, first && lane == 0);
+      const Unit U = get_unit(a, G, n_chunks, n_tiles, tpu, u, first && lane == 0);
       const int qb = it & 1;
       const uint32_t qph = (it >> 1) & 1;
       if (first) {
@@ -221,7 +225,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
       uint32_t kph = 0, aph = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-        const Unit U = get_unit(a, G, n_chunks, n_tiles, u, false);
+        const Unit U = get_unit(a, G, n_chunks, n_tiles, tpu, u, false);
         const int qb = it & 1;
         const uint32_t qph = (it >> 1) & 1;
         if (!mbar_wait(&S.q_full[qb], qph, a.status)) break;
@@ -284,8 +288,9 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
     // After a timed-out wait the warp stops waiting and computing but keeps
     // walking the same units, so every epilogue warp meets every named barrier.
     bool ok = true;
+    griddep_wait();
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-      const Unit U = get_unit(a, G, n_chunks, n_tiles, u, false);
+      const Unit U = get_unit(a, G, n_chunks, n_tiles, tpu, u, false);
       named_bar_sync(1, kEpiThreads);
       for (int i = et; i < U.ng * kHeads; i += kEpiThreads) {
         const int g = i / kHeads;
@@ -405,13 +410,34 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
 
 }  // namespace
 
-cudaError_t launch_indexer_fp8(const IndexerFp8Args& a, int num_sms, cudaStream_t stream) {
+// Tiles per work unit: the run length (at most kTilesPerUnit, at least half
+// of it) whose units spread most evenly over the persistent CTAs, counting a
+// unit's set-up as half a tile.
+int balanced_tiles_per_unit(int n_groups, int n_tiles, int num_sms) {
+  int best = kTilesPerUnit;
+  long long best_cost = -1;
+  for (int tpu = kTilesPerUnit; tpu >= kTilesPerUnit / 2; --tpu) {
+    const long long units = static_cast<long long>(n_groups) * ((n_tiles + tpu - 1) / tpu);
+    const long long grid = units < num_sms ? units : num_sms;
+    const long long per_cta = (units + grid - 1) / grid;
+    const long long cost = per_cta * (2LL * (tpu < n_tiles ? tpu : n_tiles) + 1);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = tpu;
+    }
+  }
+  return best;
+}
+
+cudaError_t launch_indexer_fp8(const IndexerFp8Args& a, int num_sms, bool pdl,
+                               cudaStream_t stream) {
   const int G = a.keys.paged ? 1 : kMaxG;
   const int n_groups = (a.qr.n_rows + G - 1) / G;
   const int n_tiles = (a.n_cols + kKeyTile - 1) / kKeyTile;
-  const int n_chunks = (n_tiles + kTilesPerUnit - 1) / kTilesPerUnit;
+  if (n_groups <= 0 || n_tiles <= 0) return cudaSuccess;
+  const int tpu = balanced_tiles_per_unit(n_groups, n_tiles, num_sms);
+  const int n_chunks = (n_tiles + tpu - 1) / tpu;
   const long long n_units_ll = static_cast<long long>(n_groups) * n_chunks;
-  if (n_units_ll <= 0) return cudaSuccess;
   if (n_units_ll > 0x7fffffffLL) return cudaErrorInvalidValue;
   const int n_units = static_cast<int>(n_units_ll);
   const size_t smem = sizeof(Smem) + 1024;
@@ -419,9 +445,17 @@ cudaError_t launch_indexer_fp8(const IndexerFp8Args& a, int num_sms, cudaStream_
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int grid = n_units < num_sms ? n_units : num_sms;
-  indexer_fp8_kernel<<<grid, kThreads, smem, stream>>>(a, G, n_chunks, n_tiles, n_units);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_units < num_sms ? n_units : num_sms);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, indexer_fp8_kernel, a, G, n_chunks, n_tiles, tpu, n_units);
 }
 
 }  // namespace dsa

@@ -219,6 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
   const int lane = tid & 31, w = tid >> 5;
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld_scores;
   int32_t* out = a.idx + static_cast<int64_t>(r) * a.ld_idx;
+  griddep_launch_dependents();
+  griddep_wait();   // the score rows come from the kernel before this one
   const int pos = a.row_pos ? a.row_pos[r] - a.pos_minus : a.pos_base + r;
   if (pos < 0 || pos >= a.ld_scores) {
     if (tid == 0) report(a.status, DSA_ERR_DEVICE_BOUNDS);
@@ -368,14 +370,23 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
 
 }  // namespace
 
-cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
+cudaError_t launch_topk(const TopkArgs& a, bool pdl, cudaStream_t stream) {
   if (a.n_rows <= 0) return cudaSuccess;
   const size_t smem = sizeof(TopkSmem);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  topk_kernel<<<a.n_rows, kThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.n_rows);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, topk_kernel, a);
 }
 
 }  // namespace dsa
