@@ -277,17 +277,33 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
   // Warp w takes scores [c0 + 256 w, c0 + 256 w + 256) of a chunk: two slices
   // of 128, lane l holding scores 4l..4l+3 of a slice (float4 rows) or, for
   // other rows, scores j*32 + l.
+  // float4 rows load the next chunk before the block scan of this one.
   const uint32_t lt = (1u << lane) - 1u;
   uint32_t base = 0;
+  float4 nxt[kPer / 4];
+  if (vec) {
+#pragma unroll
+    for (int h = 0; h < kPer / 4; ++h) {
+      const int i0 = w * (32 * kPer) + h * 128 + 4 * lane;
+      nxt[h] = i0 < n ? row4[i0 >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
   for (int c0 = 0; c0 < n; c0 += kChunk) {
     uint32_t bal[kPer], key[kPer];
     uint32_t cnt = 0;
     const int wbase = c0 + w * (32 * kPer);
     if (vec) {
+      float4 cur[kPer / 4];
+#pragma unroll
+      for (int h = 0; h < kPer / 4; ++h) {
+        cur[h] = nxt[h];
+        const int i1 = wbase + kChunk + h * 128 + 4 * lane;
+        nxt[h] = i1 < n ? row4[i1 >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
 #pragma unroll
       for (int h = 0; h < kPer / 4; ++h) {
         const int i0 = wbase + h * 128 + 4 * lane;
-        const float4 v = i0 < n ? row4[i0 >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 v = cur[h];
         key[4 * h + 0] = i0 < n ? order_key(v.x) : 0u;
         key[4 * h + 1] = i0 + 1 < n ? order_key(v.y) : 0u;
         key[4 * h + 2] = i0 + 2 < n ? order_key(v.z) : 0u;
