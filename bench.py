@@ -47,14 +47,15 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_traffic(kernel: str):
-    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None
-    when the kernel's source changed since the capture."""
+def kernel_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` on `workload` from the committed ncu
+    summary, or None when it was captured on another workload or the kernel's
+    source changed since the capture."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(kernel)
-    if not d:
+    if not d or d.get("workload") != workload:
         return None
     src = os.path.join(ROOT, "sparse_attention_long_tcgen05_b200", "csrc", d["source"])
     if not os.path.exists(src):
@@ -262,14 +263,14 @@ def run_ours(args, world, rank, local):
     }
     # The roofline is reported for the single kernel with the largest share of
     # a step: the attention kernel (one launch per step). The ncu launch list
-    # of this command at 128K gives it 46% of the step, the indexer 41% (over
-    # 1024 launches) and the top-k 12%;
+    # of this command at 128K gives it 47% of the step, the indexer 43% (over
+    # 886 launches) and the top-k 9.5%;
     # the select stage's FP8 rate is reported under "stages".
     roof = {"kernel": "sparse_mqa_bf16_kernel", "bound": "tensor", "achieved": attn_tf,
             "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
             "frac": attn_tf / peaks["bf16_sustained"],
             "peak_note": f"bf16 dense sustained ({peaks['source']})",
-            "traffic": kernel_traffic("sparse_mqa_bf16_kernel")}
+            "traffic": kernel_traffic("sparse_mqa_bf16_kernel", wl.name)}
 
     # ------------------------------------------------------------ e2e (host buffers)
     e2e = None
