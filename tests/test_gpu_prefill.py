@@ -140,7 +140,8 @@ def test_topk_heavy_ties_fallback(libs):
 def test_topk_row_layouts(libs):
     """Score rows read as float4 (16-byte aligned rows, pitch a multiple of 4)
     and rows read one score at a time (odd pitch or an unaligned first row),
-    each with ragged lengths, give the oracle's selection bit for bit."""
+    each with ragged lengths, give the oracle's selection bit for bit; rows of
+    subnormal scores put the selection threshold among the subnormals."""
     dsa, T = libs
     rng = np.random.default_rng(11)
     R, n = 24, 9000
@@ -149,6 +150,11 @@ def test_topk_row_layouts(libs):
     for pitch, offset in ((9000, 0), (9004, 0), (9003, 0), (9004, 1), (9001, 3)):
         buf = torch.from_numpy(rng.standard_normal(R * pitch + offset).astype(np.float32))
         buf[offset:].view(R, pitch)[:, :n:7] = 2.5          # ties around the k-th score
+        rows = buf[offset:].view(R, pitch)
+        rows[4] *= 1e-41                                    # subnormal scores only
+        rows[5] = -rows[5].abs() * 1e-42                    # negative subnormals and zeros
+        rows[5, ::5] = 0.0
+        rows[5, 1::5] = -0.0
         s = buf.cuda()[offset:offset + R * pitch].view(R, pitch)[:, :n]
         for k in (2048, 33):
             idx = torch.empty(R, k, dtype=torch.int32, device="cuda")
