@@ -17,7 +17,7 @@
 // with keys on TMEM lanes and (query, head) on TMEM columns, so each epilogue
 // thread owns one key and reduces the 64 heads of a query inside its registers.
 //
-// Roles (320 threads, one CTA per SM, persistent over work units):
+// Roles (352 threads, one CTA per SM, persistent over work units):
 //   warp 0    TMA producer: Q group (once per unit), key tiles and their fp32
 //             key scales through a 6-stage ring; in paged mode it loads the
 //             first 64-key page of each tile and warp 10 the second (a TMA
@@ -31,7 +31,12 @@
 //             two key tiles, one per 64-column half of a 128-column
 //             accumulator, and warps 2-5 reduce the first, warps 6-9 the
 //             second, so both halves of the epilogue work.
-// A work unit is (group of G query rows, run of up to 16 key tiles of 128).
+//   warp 10   second paged producer (idle on contiguous keys)
+// A work unit is (group of G query rows, run of 8..16 key tiles of 128); the
+// launcher picks the run length that spreads the units most evenly over the
+// CTAs. Launched after another kernel of the same selection, the kernel
+// starts at once and only the epilogue, which overwrites the score rows that
+// kernel may still read, waits for it (griddepcontrol).
 #include "dsa_common.cuh"
 #include "dsa_kernels.h"
 #include "indexer_epilogue.cuh"
