@@ -127,17 +127,24 @@ class Clocks:
                 "power_w_max": max((num(r[3]) or 0) for r in loaded)}
 
 
+def dist_env():
+    """(world, rank, local rank) from the launcher's environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
 def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    """One process per GPU: NCCL over the node's GPUs, or gloo on a host
+    without one (the host logic below is the same)."""
+    world, rank, local = dist_env()
+    cuda = torch.cuda.is_available()
+    if cuda:
+        torch.cuda.set_device(local)
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                             device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(local)
+        kw = {"device_id": torch.device("cuda", local)} if cuda else {}
+        torch.distributed.init_process_group("nccl" if cuda else "gloo",
+                                             timeout=datetime.timedelta(seconds=300), **kw)
     return world, rank, local
 
 
@@ -149,9 +156,16 @@ def barrier(world):
 def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: every rank processes `units_per_rank` in a step,
+    the step takes `ms` on the slowest rank."""
+    return world * units_per_rank / (ms * 1e-3)
 
 
 def timed(fn, steps, warmup, world, pre=None):
@@ -285,7 +299,7 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.skip_cpu:
         cpu = oracle_prefill_rate(inp, wl, budget_s=args.cpu_budget)
 
-    value_tok = world * L / (ms * 1e-3)
+    value_tok = job_rate(world, L, ms)
     res = {
         "metric": METRIC, "value": value_tok, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -325,7 +339,7 @@ def prefill_e2e(dsa, inp, ind, att, ws, idx, out, lse, k, args, world):
     ms = timed(step, args.e2e_steps, 1, world)
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * 4
-    return {"value": world * inp.wl.L / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+    return {"value": job_rate(world, inp.wl.L, ms), "unit": "tokens/s", "ms_per_step": ms,
             "steps": args.e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
@@ -418,11 +432,11 @@ def run_decode(args, world, rank, local, peaks, dsa, make_decode, wl):
             fwd()
             host_out.copy_(out, non_blocking=True)
         ms_e2e = timed(step, steps, 1, world, pre=flush)
-        e2e = {"value": world * B / (ms_e2e * 1e-3), "unit": "tokens/s", "ms_per_step": ms_e2e,
+        e2e = {"value": job_rate(world, B, ms_e2e), "unit": "tokens/s", "ms_per_step": ms_e2e,
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host_in),
                "d2h_bytes_per_step": host_out.numel() * host_out.element_size()}
     return {
-        "workload": wl.name, "value": world * B / (ms * 1e-3), "unit": "tokens/s",
+        "workload": wl.name, "value": job_rate(world, B, ms), "unit": "tokens/s",
         "ms_per_step": ms, "steps": steps, "l2": "flushed before every step (untimed)",
         "mean_ctx": float(ctx.float().mean()),
         "roofline": {"kernel": "whole decode step", "bound": "hbm", "achieved": step_gbs,
@@ -484,13 +498,15 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    world, rank, local = dist_setup() if torch.cuda.is_available() else (1, 0, 0)
     if args.impl == "reference":
+        # the oracle on the host cores: rank 0 alone, no process group
+        world, rank, _ = dist_env()
         if rank != 0:
             return
-        res = run_reference(args, world, rank)
-    else:
-        res = run_ours(args, world, rank, local)
+        print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return
+    world, rank, local = dist_setup()
+    res = run_ours(args, world, rank, local)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:
