@@ -313,12 +313,15 @@ def test_forward_L4096(libs):
     _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, sample_rows(L, 64, seed=1))
 
 
-def test_forward_two_score_blocks_L5000(libs):
-    """A prefill whose scores do not fit one block (4144 rows, then a ragged
-    856): the fused selection equals the standalone top-k of the standalone
-    scores in every row."""
+@pytest.mark.parametrize("L", [5000, 16384])
+def test_forward_score_blocks_every_row(libs, L):
+    """Prefills whose scores span several blocks (5000: 4144 rows, then a ragged
+    856; 16384: 13 blocks of 1184 rows and a ragged 992), so each indexer launch
+    after the first overwrites the block the previous top-k reads: the fused
+    selection equals the standalone top-k of the standalone scores in every
+    row."""
     dsa, T = libs
-    inp = make_prefill(_wl(5000), device="cuda", seed=3)
+    inp = make_prefill(_wl(L), device="cuda", seed=3)
     ind, att, idx, out, lse = _forward(dsa, T, inp)
     L, k = inp.wl.L, inp.wl.k
     scores = torch.empty(L, L, device="cuda")
