@@ -146,14 +146,7 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   return r;
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                              uint32_t d) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b),
-               "r"(c), "r"(d)
-               : "memory");
-}
-
-// Asynchronous 16-byte store into a peer CTA's shared memory that counts its
+// Asynchronous 4-byte store into a peer CTA's shared memory that counts its
 // bytes on the peer's mbarrier (complete_tx) when it lands: the peer's wait on
 // that barrier makes the data visible without any fence on this side.
 __device__ __forceinline__ void st_async_b32(uint32_t cluster_addr, uint32_t v,
@@ -165,18 +158,9 @@ __device__ __forceinline__ void st_async_b32(uint32_t cluster_addr, uint32_t v,
       : "memory");
 }
 
-__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t a, uint32_t b,
-                                            uint32_t c, uint32_t d, uint32_t cluster_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, "
-      "[%5];" ::"r"(cluster_addr),
-      "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_bar)
-      : "memory");
-}
-
 // Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from
 // this CTA's shared memory into a peer CTA's, counted on the peer's mbarrier
-// (complete_tx). One asynchronous operation instead of bytes / 16 st.async.
+// (complete_tx). One asynchronous operation for the whole range.
 // Generic-proxy writes to the source must be fenced (fence_proxy_async_smem)
 // before the copy is issued.
 __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint32_t src_cta,
@@ -194,13 +178,6 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint3
 // consumes every value it loaded, issued before the arrive).
 __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_bar_addr) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                   cluster_bar_addr)
-               : "memory");
-}
-
-// Arrive (release at cluster scope) on an mbarrier that may live in the peer CTA.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
                    cluster_bar_addr)
                : "memory");
 }
@@ -260,18 +237,6 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
       "r"(y2), "r"(y3)
       : "memory");
-}
-
-// 16-byte global -> shared copy (L2 only), completion tracked per thread.
-__device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
-}
-
-// One arrival on `bar` once every cp.async this thread issued so far has landed
-// (the arrival is one of the barrier's expected arrivals).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05 / TMEM
@@ -473,8 +438,6 @@ __device__ __forceinline__ void regs_dec() {
 }
 
 // ------------------------------------------------------------------ misc
-
-__device__ __forceinline__ uint32_t elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
