@@ -20,7 +20,12 @@
  *     the caller's workspace, sized by dsa_workspace_size().
  *   - Every call is asynchronous on the given CUDA stream (a cudaStream_t;
  *     NULL is the legacy default stream). Host-side argument checks run before
- *     any launch and return an error without launching anything.
+ *     any launch and return an error without launching anything. A call's
+ *     first kernel starts after all earlier work on the stream; inside one
+ *     dsa_select / dsa_forward the indexer and top-k launches may overlap one
+ *     another's start-up (programmatic dependent launch), never their reads
+ *     and writes of shared buffers, and the work after the call sees all of
+ *     its results. Streams captured into CUDA graphs keep these rules.
  *   - Errors found on the device (an index or page id out of range, a bounded
  *     wait that ran out) are recorded in a per-device status word; read it
  *     with dsa_check_status(), which synchronises the stream. Device code
