@@ -25,7 +25,7 @@
  *     dsa_select / dsa_forward the indexer and top-k launches may overlap one
  *     another's start-up (programmatic dependent launch), never their reads
  *     and writes of shared buffers, and the work after the call sees all of
- *     its results. Streams captured into CUDA graphs keep these rules.
+ *     its results.
  *   - Errors found on the device (an index or page id out of range, a bounded
  *     wait that ran out) are recorded in a per-device status word; read it
  *     with dsa_check_status(), which synchronises the stream. Device code
