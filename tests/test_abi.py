@@ -59,6 +59,17 @@ def test_workspace_size_host_logic(lib):
     idx_bytes = L * 2048 * 4
     assert idx_bytes < nbytes <= idx_bytes + (80 << 20) + 512
     assert lib.dsa_workspace_size(lib.DSA_OP_SPARSE_MQA) == 0
+    # the score block: whole waves of 148 top-k CTAs within 80 MiB, or the
+    # whole prefill when it fits
+    for n in (4096, 32768, 65536, 131072):
+        qn = torch.empty(n, 64, 128, dtype=torch.uint8)
+        kn = torch.empty(n, 128, dtype=torch.uint8)
+        sn = torch.empty(n)
+        indn = lib.indexer_in(qn, kn, torch.empty(n, 64), sn, sn)
+        sel = lib.dsa_workspace_size(lib.DSA_OP_SELECT, indn, None, 0, 0, 2048)
+        rows = sel // (n * 4)
+        assert sel - rows * n * 4 < 256 and rows * n * 4 <= (80 << 20)
+        assert rows == n if n * n * 4 <= (80 << 20) else rows % 148 == 0
     with pytest.raises(lib.DsaError):
         lib.dsa_workspace_size(lib.DSA_OP_FORWARD, ind, None, 0, 0, 4096)   # k > 2048
 
