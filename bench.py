@@ -47,6 +47,53 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
+def measure_fp8_peak(n=8192, reps=10, sustain_s=3.0):
+    """Dense FP8 (e4m3 x e4m3 -> bf16, f32 accumulate) tensor throughput of this
+    GPU, measured with the library GEMM torch._scaled_mm on n^3 (2 n^3 flops):
+    best of `reps` single calls (burst) and ~sustain_s seconds of calls back to
+    back (sustained, the figure for a kernel timed inside a long step). Both
+    the default and the fast-accumulation GEMM are tried; the faster counts."""
+    a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()   # column-major
+    one = torch.ones((), device="cuda")
+    flops = 2.0 * n ** 3
+    best = {}
+    for fast in (False, True):
+        def mm():
+            return torch._scaled_mm(a, b, one, one, out_dtype=torch.bfloat16,
+                                    use_fast_accum=fast)
+        for _ in range(3):
+            mm()
+        torch.cuda.synchronize()
+        t = []
+        for _ in range(reps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            mm()
+            e1.record()
+            torch.cuda.synchronize()
+            t.append(e0.elapsed_time(e1))
+        burst_ms = min(t)
+        iters = max(10, int(sustain_s * 1e3 / burst_ms))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            mm()
+        e1.record()
+        torch.cuda.synchronize()
+        sus_ms = e0.elapsed_time(e1) / iters
+        best[fast] = (flops / (burst_ms * 1e-3) / 1e12, flops / (sus_ms * 1e-3) / 1e12)
+    fast = max(best, key=lambda f: best[f][0])
+    del a, b
+    torch.cuda.empty_cache()
+    return {"fp8_tflops": best[fast][0], "fp8_tflops_sustained": best[fast][1],
+            "how": f"torch._scaled_mm e4m3 {n}^3, bf16 out, use_fast_accum={fast}: best of "
+                   f"{reps} (burst) and ~{sustain_s:.0f} s back to back (sustained)",
+            "default_accum_tflops": best[False][0], "fast_accum_tflops": best[True][0]}
+
+
 def kernel_traffic(kernel: str, workload: str):
     """Per-launch DRAM bytes of `kernel` on `workload` from the committed ncu
     summary, or None when it was captured on another workload or the kernel's
@@ -229,10 +276,14 @@ def run_ours(args, world, rank, local):
     from sparse_attention_long_tcgen05_b200.inputs import WORKLOADS, make_prefill, make_decode
 
     peaks = load_peaks()
-    fp8_sustained = 2.0 * peaks["bf16_sustained"]   # FP8 dense = 2x bf16 (nominal ratio)
     if args.decode_only:    # profiling aid: the decode step alone
-        return {"decode": run_decode(args, world, rank, local, peaks, dsa, make_decode,
-                                     WORKLOADS[DECODE_WL])}
+        dwl = WORKLOADS[DECODE_WL]
+        if args.decode_ctx_max:
+            import dataclasses
+            dwl = dataclasses.replace(dwl, name=f"decode_B64_ctx{args.decode_ctx_max}",
+                                      ctx_min=min(dwl.ctx_min, args.decode_ctx_max // 2),
+                                      ctx_max=args.decode_ctx_max)
+        return {"decode": run_decode(args, world, rank, local, peaks, dsa, make_decode, dwl)}
     wl = next(w for w in WORKLOADS.values() if w.name == args.workload)
     L, k = wl.L, wl.k
     inp = make_prefill(wl, device="cuda", seed=rank)
@@ -252,6 +303,20 @@ def run_ours(args, world, rank, local):
     def attn():
         dsa.dsa_sparse_mqa_fwd(att, idx, k, out, lse)
 
+    # the indexer alone, launched over the same blocks of query rows as the
+    # fused selection (each block's rows against keys 0..last row of the block)
+    sel_bytes = dsa.dsa_workspace_size(dsa.DSA_OP_SELECT, ind, None, 0, 0, k)
+    chunk = max(1, min(L, sel_bytes // (L * 4)))
+    rows_all = torch.arange(L, dtype=torch.int32, device="cuda")
+    blocks = [(q0, min(chunk, L - q0)) for q0 in range(0, L, chunk)]
+    ws_f = ws[: (sel_bytes // 4) * 4].view(torch.float32)
+
+    def indexer_alone():
+        for q0, rows in blocks:
+            cols = q0 + rows
+            dsa.dsa_indexer_scores(ind, rows_all[q0:q0 + rows], rows,
+                                   ws_f[: rows * cols].view(rows, cols), cols)
+
     with Clocks(local) as clk:
         n0 = dsa.dsa_launch_counter()
         ms = timed(fwd, args.steps, args.warmup, world)
@@ -263,28 +328,49 @@ def run_ours(args, world, rank, local):
     per_call = launches / (args.steps + args.warmup)
     ms_sel = timed(sel, args.steps, 1, world)
     ms_attn = timed(attn, args.steps, 1, world)
+    ms_idx = timed(indexer_alone, args.steps, 1, world)
+    st = dsa.dsa_check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {dsa.status_string(st)}")
+    fp8 = measure_fp8_peak() if not args.skip_fp8_peak else None
+    fp8_sus = fp8["fp8_tflops_sustained"] if fp8 else 2.0 * peaks["bf16_sustained"]
+    fp8_note = ("FP8 dense sustained, measured in this run (torch._scaled_mm)" if fp8 else
+                f"2 x bf16 dense sustained ({peaks['source']}; nominal FP8/bf16 ratio)")
 
     idx_flops = 2.0 * wl.H_I * wl.d_I * (L * (L + 1) / 2)
     attn_flops = 2.0 * wl.H * (wl.D_K + wl.D_V) * attention_pairs(L, k)
+    idx_tf = idx_flops / (ms_idx * 1e-3) / 1e12
     sel_tf = idx_flops / (ms_sel * 1e-3) / 1e12
     attn_tf = attn_flops / (ms_attn * 1e-3) / 1e12
     stages = {
         "select_ms": ms_sel, "select_fp8_tflops": sel_tf,
-        "select_frac_fp8_sustained": sel_tf / fp8_sustained,
+        "indexer_ms": ms_idx, "indexer_launches": len(blocks), "indexer_rows_per_launch": chunk,
+        "indexer_fp8_tflops": idx_tf,
+        "indexer_frac_fp8_sustained": idx_tf / fp8_sus,
+        "indexer_frac_fp8_nominal_2x_bf16_sustained": idx_tf / (2.0 * peaks["bf16_sustained"]),
+        "topk_ms_estimate": ms_sel - ms_idx,
         "attention_ms": ms_attn, "attention_bf16_tflops": attn_tf,
         "attention_frac_bf16_sustained": attn_tf / peaks["bf16_sustained"],
         "indexer_flops": idx_flops, "attention_flops": attn_flops,
     }
-    # The roofline is reported for the single kernel with the largest share of
-    # a step: the attention kernel (one launch per step). The ncu launch list
-    # of this command at 128K gives it 47% of the step, the indexer 43% (over
-    # 886 launches) and the top-k 9.5%;
-    # the select stage's FP8 rate is reported under "stages".
-    roof = {"kernel": "sparse_mqa_bf16_kernel", "bound": "tensor", "achieved": attn_tf,
-            "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-            "frac": attn_tf / peaks["bf16_sustained"],
+    rooflines = {
+        "indexer_fp8_kernel": {
+            "bound": "tensor", "achieved": idx_tf, "peak": fp8_sus, "unit": "TFLOP/s",
+            "frac": idx_tf / fp8_sus, "peak_note": fp8_note,
+            "algorithmic": "2*64*128 FP8 flops per (t, s<=t) pair, L(L+1)/2 pairs",
+            "launches": len(blocks), "ms": ms_idx,
+            "traffic": kernel_traffic("indexer_fp8_kernel", wl.name)},
+        "sparse_mqa_bf16_kernel": {
+            "bound": "tensor", "achieved": attn_tf, "peak": peaks["bf16_sustained"],
+            "unit": "TFLOP/s", "frac": attn_tf / peaks["bf16_sustained"],
             "peak_note": f"bf16 dense sustained ({peaks['source']})",
-            "traffic": kernel_traffic("sparse_mqa_bf16_kernel", wl.name)}
+            "algorithmic": "2*128*(576+512) bf16 flops per selected (t, key) pair",
+            "launches": 1, "ms": ms_attn,
+            "traffic": kernel_traffic("sparse_mqa_bf16_kernel", wl.name)},
+    }
+    # the headline roofline is that of the kernel with the largest share of the step
+    dom = "indexer_fp8_kernel" if ms_idx > ms_attn else "sparse_mqa_bf16_kernel"
+    roof = dict(rooflines[dom], kernel=dom)
 
     # ------------------------------------------------------------ e2e (host buffers)
     e2e = None
@@ -309,7 +395,8 @@ def run_ours(args, world, rank, local):
                    "H": wl.H, "d_qk": wl.D_K, "d_v": wl.D_V, "seed": "rank",
                    "l2": "inputs larger than L2 (q alone 19.3 GB)",
                    "parallelism": f"replicas x{world} (independent sequences)"},
-        "roofline": roof, "stages": stages, "cpu_baseline": cpu, "e2e": e2e,
+        "roofline": roof, "rooflines": rooflines, "fp8_peak": fp8, "stages": stages,
+        "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": int(round(per_call * args.steps)),
         "clocks": clk.summary(),
     }
@@ -321,26 +408,64 @@ def run_ours(args, world, rank, local):
     return res
 
 
-def prefill_e2e(dsa, inp, ind, att, ws, idx, out, lse, k, args, world):
-    """Same metric through the public call with host buffers: every step copies
-    its inputs from pinned host memory and reads the attention output back."""
-    dev_in = [inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.q, inp.kv]
-    host_in = [pinned_copy(t) for t in dev_in]
+def prefill_e2e(dsa, inp, ind, att, ws, idx, out, lse, k, args, world, n_chunks=8):
+    """Same metric through the public calls with HOST buffers: every step copies
+    all of its inputs from pinned host memory and reads the attention output and
+    lse back, and the copies overlap the kernels. The indexer-side inputs and the
+    latent cache go up first; q (19.3 GB at 128K) streams up in n_chunks row
+    chunks on a copy stream while dsa_select runs; dsa_sparse_mqa_fwd then runs
+    chunk by chunk as each chunk's q lands (the chunk's queries are the suffix
+    of the first c1 keys, so positions are unchanged), and each chunk's output
+    goes back on a second copy stream while the next chunk computes."""
+    wl = inp.wl
+    L = wl.L
+    small = [inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.kv]
+    host_small = [pinned_copy(t) for t in small]
+    host_q = pinned_copy(inp.q)
     host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    bounds = [(L * c // n_chunks, L * (c + 1) // n_chunks) for c in range(n_chunks)]
+    atts = [dsa.attn_in(inp.q[c0:c1], inp.kv[:c1], wl.scale, wl.D_V) for c0, c1 in bounds]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
     def step():
-        for h, d in zip(host_in, dev_in):
-            d.copy_(h, non_blocking=True)
-        dsa.dsa_forward(ind, att, k, idx, out, lse, ws)
-        host_out.copy_(out, non_blocking=True)
-        host_lse.copy_(lse, non_blocking=True)
+        comp = torch.cuda.current_stream()
+        go = torch.cuda.Event()
+        go.record(comp)
+        ev_small, ev_q, ev_o = torch.cuda.Event(), [], []
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(go)
+            for h, d in zip(host_small, small):
+                d.copy_(h, non_blocking=True)
+            ev_small.record(s_in)
+            for c0, c1 in bounds:
+                inp.q[c0:c1].copy_(host_q[c0:c1], non_blocking=True)
+                ev_q.append(torch.cuda.Event())
+                ev_q[-1].record(s_in)
+        comp.wait_event(ev_small)
+        dsa.dsa_select(ind, k, idx, ws)
+        for c, (c0, c1) in enumerate(bounds):
+            comp.wait_event(ev_q[c])
+            dsa.dsa_sparse_mqa_fwd(atts[c], idx[c0:c1], k, out[c0:c1], lse[c0:c1])
+            ev_o.append(torch.cuda.Event())
+            ev_o[-1].record(comp)
+        with torch.cuda.stream(s_out):
+            for c, (c0, c1) in enumerate(bounds):
+                s_out.wait_event(ev_o[c])
+                host_out[c0:c1].copy_(out[c0:c1], non_blocking=True)
+                host_lse[c0:c1].copy_(lse[c0:c1], non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(s_out)
+        comp.wait_event(done)
 
     ms = timed(step, args.e2e_steps, 1, world)
-    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    h2d = sum(t.numel() * t.element_size() for t in host_small) + \
+        host_q.numel() * host_q.element_size()
     d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * 4
-    return {"value": job_rate(world, inp.wl.L, ms), "unit": "tokens/s", "ms_per_step": ms,
-            "steps": args.e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    return {"value": job_rate(world, L, ms), "unit": "tokens/s", "ms_per_step": ms,
+            "steps": args.e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "how": f"pinned host buffers; dsa_select + {n_chunks} chunked dsa_sparse_mqa_fwd "
+                   "calls, host<->device copies on two copy streams overlapping the kernels"}
 
 
 def oracle_prefill_rate(inp, wl, budget_s=15.0, rows_cap=None):
@@ -442,6 +567,24 @@ def run_decode(args, world, rank, local, peaks, dsa, make_decode, wl):
         "roofline": {"kernel": "whole decode step", "bound": "hbm", "achieved": step_gbs,
                      "peak": hbm, "unit": "GB/s", "frac": step_gbs / hbm,
                      "algorithmic_bytes_per_step": step_bytes, "traffic": None},
+        "rooflines": {
+            # the sparse gather: every selected latent row once (1152 B) + q in, O out
+            "sparse_mqa_bf16_kernel": {
+                "bound": "hbm", "achieved": attn_gbs, "peak": hbm, "unit": "GB/s",
+                "frac": attn_gbs / hbm, "ms": ms_attn,
+                "algorithmic_bytes": gather_bytes + B * (wl.H * wl.D_K * 2 + wl.H * wl.D_V * 2),
+                "algorithmic": "sum_b min(k, ctx_b) * 1152 B + q (147 KB) + O (131 KB) per "
+                               "sequence",
+                "traffic": kernel_traffic("sparse_mqa_bf16_kernel", wl.name)},
+            # the key-cache scan of the indexer (+ its top-k): every cached key's
+            # e4m3 row and scale once, q_I and w in
+            "select (indexer_fp8_kernel + topk_kernel)": {
+                "bound": "hbm", "achieved": sel_gbs, "peak": hbm, "unit": "GB/s",
+                "frac": sel_gbs / hbm, "ms": ms_sel,
+                "algorithmic_bytes": scan_bytes + B * (wl.H_I * wl.d_I + wl.H_I * 4),
+                "algorithmic": "sum_b ctx_b * 132 B + q_I (8 KB) + w (256 B) per sequence",
+                "traffic": kernel_traffic("indexer_fp8_kernel", wl.name)},
+        },
         "stages": {"select_ms": ms_sel, "select_gbs": sel_gbs, "select_frac_hbm": sel_gbs / hbm,
                    "attention_ms": ms_attn, "attention_gbs": attn_gbs,
                    "attention_frac_hbm": attn_gbs / hbm},
@@ -490,9 +633,15 @@ def main():
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the decode step (profiling aid; no headline value)")
+    ap.add_argument("--decode-ctx-max", type=int, default=0,
+                    help="with --decode-only: a smaller decode (context lengths up to this) "
+                         "for multi-pass profiling")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--skip-fp8-peak", action="store_true",
+                    help="do not measure the FP8 GEMM peak (the indexer is then reported "
+                         "against 2 x the bf16 peak)")
+    ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=10.0)
     args = ap.parse_args()

@@ -17,26 +17,32 @@
  * Conventions shared by every call
  *   - Every tensor pointer is a DEVICE pointer owned by the caller. The
  *     library never allocates device memory on these paths; scratch space is
- *     the caller's workspace, sized by dsa_workspace_size().
+ *     the caller's workspace, sized by dsa_workspace_size(). The one
+ *     exception is dsa_select_noalloc, which takes no workspace and keeps its
+ *     score rows in a fixed 16 MiB scratch array that the library holds on
+ *     each GPU that loads it (see its declaration).
  *   - Every call is asynchronous on the given CUDA stream (a cudaStream_t;
  *     NULL is the legacy default stream). Host-side argument checks run before
  *     any launch and return an error without launching anything. A call's
  *     first kernel starts after all earlier work on the stream; inside one
- *     dsa_select / dsa_forward the indexer and top-k launches may overlap one
- *     another's start-up (programmatic dependent launch), never their reads
- *     and writes of shared buffers, and the work after the call sees all of
- *     its results.
+ *     dsa_select / dsa_select_noalloc / dsa_forward the indexer and top-k
+ *     launches may overlap one another's start-up (programmatic dependent
+ *     launch), never their reads and writes of shared buffers, and the work
+ *     after the call sees all of its results.
  *   - Errors found on the device (an index or page id out of range, a bounded
  *     wait that ran out) are recorded in a per-device status word; read it
  *     with dsa_check_status(), which synchronises the stream. Device code
  *     never traps: bad indices are skipped (treated as masked) and reported.
  *   - Positions. CONTIGUOUS layout: keys are rows 0..n_keys-1 of one
  *     sequence and query i sits at position n_keys - n_q + i (n_q == n_keys is
- *     a plain prefill). PAGED layout: query b belongs to sequence b, whose
- *     ctx_lens[b] cached tokens include the query token, so the query sits at
- *     position ctx_lens[b] - 1. In both cases the query sees keys 0..pos
- *     (inclusive: the pages say "preceding tokens"; the token itself is kept so
- *     that every row has at least one key).
+ *     a plain prefill; n_q < n_keys is a chunk of a longer prefill). PAGED
+ *     layout: query i belongs to sequence b = q_seq ? q_seq[i] : i, whose
+ *     ctx_lens[b] cached tokens include the query's own, and sits at position
+ *     q_pos ? q_pos[i] : ctx_lens[b] - 1. In both cases the query sees keys
+ *     0..pos of its sequence (inclusive: the pages say "preceding tokens"; the
+ *     token itself is kept so that every row has at least one key). A query
+ *     whose sequence, length or position is out of range is reported as
+ *     DSA_ERR_DEVICE_BOUNDS and gets an empty selection.
  *   - Supported combinations (others return DSA_ERR_UNSUPPORTED):
  *       E4M3 indexer (H_I=64, d_I=128) + BF16 attention (H=128, d_qk=576,
  *       d_v=512, V = first 512 columns of the KV row), CONTIGUOUS or PAGED
@@ -85,15 +91,22 @@ typedef enum dsa_kv_kind {
 } dsa_kv_kind;
 
 /* Where the keys live. For PAGED, logical token p of sequence b is slot
- * p % page_size of page block_table[b * ld_block_table + p / page_size]. */
+ * p % page_size of page block_table[b * ld_block_table + p / page_size].
+ * A PAGED query belongs to one sequence and sits at one position in it (see
+ * "Positions" above): with q_seq and q_pos NULL, query b is the newest token
+ * of sequence b (decode); with them, several queries may share a sequence
+ * (multi-token decode, a chunk of a prefill against the paged cache). */
 typedef struct dsa_kv_layout {
   int32_t kind;                 /* dsa_kv_kind */
   int32_t page_size;            /* PAGED: tokens per page, must be 64 */
-  const int32_t* block_table;   /* PAGED: device [n_q, ld_block_table] page ids */
+  const int32_t* block_table;   /* PAGED: device [n_seq, ld_block_table] page ids */
   int64_t ld_block_table;       /* PAGED: elements between rows of block_table */
   int32_t max_pages;            /* PAGED: columns of block_table usable per row */
   int32_t num_pages;            /* PAGED: pages in the caches (page ids must be < this) */
-  const int32_t* ctx_lens;      /* PAGED: device [n_q] cached tokens per sequence, in [1, max_pages*page_size] */
+  const int32_t* ctx_lens;      /* PAGED: device [n_seq] cached tokens per sequence, in [1, max_pages*page_size] */
+  const int32_t* q_seq;         /* PAGED, nullable: device [n_q] sequence of each query, in [0, n_seq) (NULL: query b -> sequence b) */
+  const int32_t* q_pos;         /* PAGED, nullable: device [n_q] position of each query in its sequence, in [0, ctx_lens[seq]) (NULL: ctx_lens[seq] - 1) */
+  int32_t n_seq;                /* PAGED: sequences (rows of block_table, entries of ctx_lens); 0 means n_q. Without q_seq, n_seq >= n_q */
 } dsa_kv_layout;
 
 /* Indexer inputs (step 1). Token-major rows; all strides in ELEMENTS.
@@ -150,7 +163,8 @@ typedef enum dsa_op {
  * are written: the score for keys s <= pos(query), -INFINITY for s > pos.
  * Scores are float32 and bit-identical to those the fused dsa_forward ranks.
  * Requires n_cols >= 1, ld_scores >= n_cols; for PAGED n_cols <=
- * max_pages*page_size. Workspace: dsa_workspace_size(DSA_OP_INDEXER_SCORES). */
+ * max_pages*page_size. ws / ws_bytes are reserved and unused by this version
+ * (dsa_workspace_size(DSA_OP_INDEXER_SCORES) is 0): pass NULL / 0. */
 DSA_API dsa_status dsa_indexer_scores(const dsa_indexer_in* in, const int32_t* rows,
                                       int32_t n_rows, float* scores, int64_t ld_scores,
                                       int32_t n_cols, void* ws, size_t ws_bytes,
@@ -172,7 +186,8 @@ DSA_API dsa_status dsa_topk(const float* scores, int64_t ld_scores, const int32_
  * DSA_ERR_DEVICE_BOUNDS and skipped. Every row must hold at least one valid
  * entry. out: [n_q, heads, d_v] contiguous, same dtype as q; lse: [n_q, heads]
  * float32 natural-log log-sum-exp of the scaled logits (may be NULL).
- * Workspace: dsa_workspace_size(DSA_OP_SPARSE_MQA). */
+ * ws / ws_bytes are reserved and unused by this version
+ * (dsa_workspace_size(DSA_OP_SPARSE_MQA) is 0): pass NULL / 0. */
 DSA_API dsa_status dsa_sparse_mqa_fwd(const dsa_attn_in* in, const int32_t* idx, int64_t ld_idx,
                                       int32_t k, void* out, float* lse, void* ws,
                                       size_t ws_bytes, dsa_stream_t stream);
@@ -181,7 +196,9 @@ DSA_API dsa_status dsa_sparse_mqa_fwd(const dsa_attn_in* in, const int32_t* idx,
  * bounded blocks of queries so the n_q x n_keys score matrix never exists.
  * idx: [n_q, ld_idx] int32 (ld_idx >= k), same contents and rules as
  * dsa_topk(dsa_indexer_scores(...)) bit for bit.
- * Workspace: dsa_workspace_size(DSA_OP_SELECT). */
+ * Workspace: dsa_workspace_size(DSA_OP_SELECT): one block of float32 score
+ * rows, min(n_q, max(128, rows that fit in 80 MiB)) rows of n_keys (CONTIGUOUS)
+ * or max_pages*page_size (PAGED) columns, so it does not grow with n_q. */
 DSA_API dsa_status dsa_select(const dsa_indexer_in* indexer, int32_t k, int32_t* idx,
                               int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
@@ -237,6 +254,19 @@ DSA_API int32_t dsa_last_cuda_error(void);
 #define DSA_NOALLOC_SCRATCH_BYTES (16u << 20)
 DSA_API dsa_status dsa_select_noalloc(const dsa_indexer_in* indexer, int32_t k, int32_t* idx,
                                       int64_t ld_idx, dsa_stream_t stream);
+
+/* Failure detection: every wait inside the kernels (on a TMA copy, an MMA, a
+ * peer CTA) is bounded; a wait that runs out records DSA_ERR_TIMEOUT in the
+ * device status word (read it with dsa_check_status), the waiting role gives
+ * up, the kernel lets the copies and MMAs it already issued complete, frees its
+ * tensor memory and returns -- the GPU context stays usable, but the results of
+ * that call are invalid. No legitimate wait lasts more than microseconds.
+ * This sets the bound of the lightning-indexer kernel's pipeline waits for
+ * launches issued after the call (process-wide, all devices); ns <= 0 restores
+ * the default of 1 second. The other kernels keep the 1 s bound. A bound far
+ * below the copies' latency makes the indexer give up on purpose, which is
+ * how the failure path is tested. */
+DSA_API dsa_status dsa_set_wait_limit_ns(int64_t ns);
 
 /* Number of kernel launches this process has issued through the library so
  * far (all devices, all threads). Lets a caller count launches in a region. */

@@ -22,6 +22,10 @@ namespace {
 thread_local int32_t t_last_cuda_error = 0;
 std::atomic<int64_t> g_launches{0};
 
+// Bound of each pipeline wait of the indexer kernel (dsa_set_wait_limit_ns).
+constexpr int64_t kDefaultWaitNs = 1000LL * 1000LL * 1000LL;
+std::atomic<int64_t> g_wait_ns{kDefaultWaitNs};
+
 constexpr int kMaxDevices = 64;
 constexpr int kKMax = 2048;
 constexpr int kPage = 64;
@@ -136,9 +140,11 @@ dsa_status check_layout(const dsa_kv_layout& kv, int32_t n_q, int32_t n_keys) {
   if (kv.kind != DSA_KV_PAGED) return DSA_ERR_INVALID_ARG;
   if (kv.page_size != kPage) return DSA_ERR_UNSUPPORTED;
   if (n_q < 1 || kv.block_table == nullptr || kv.ctx_lens == nullptr || kv.max_pages < 1 ||
-      kv.num_pages < 1 || kv.ld_block_table < kv.max_pages)
+      kv.num_pages < 1 || kv.ld_block_table < kv.max_pages || kv.n_seq < 0)
     return DSA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(kv.max_pages) * kPage > 0x7fffffffLL) return DSA_ERR_INVALID_ARG;
+  // without q_seq, query b is sequence b: there must be a sequence per query
+  if (kv.q_seq == nullptr && kv.n_seq != 0 && kv.n_seq < n_q) return DSA_ERR_INVALID_ARG;
   return DSA_OK;
 }
 
@@ -152,6 +158,9 @@ dsa::KeySide key_side(const dsa_kv_layout& kv, int32_t n_q, int32_t n_keys) {
   k.max_pages = kv.max_pages;
   k.num_pages = kv.num_pages;
   k.ctx_lens = kv.ctx_lens;
+  k.q_seq = kv.q_seq;
+  k.q_pos = kv.q_pos;
+  k.n_seq = kv.n_seq > 0 ? kv.n_seq : n_q;
   return k;
 }
 
@@ -240,13 +249,8 @@ struct ForwardPlan {
 
 ForwardPlan forward_plan(const dsa_indexer_in& ind, int32_t k) {
   ForwardPlan p{};
-  if (ind.kv.kind == DSA_KV_PAGED) {
-    p.n_cols = ind.kv.max_pages * kPage;
-    p.chunk = ind.n_q;
-  } else {
-    p.n_cols = ind.n_keys;
-    p.chunk = forward_chunk_rows(ind.n_q, ind.n_keys);
-  }
+  p.n_cols = ind.kv.kind == DSA_KV_PAGED ? ind.kv.max_pages * kPage : ind.n_keys;
+  p.chunk = forward_chunk_rows(ind.n_q, p.n_cols);
   p.scores_bytes = round256(static_cast<size_t>(p.chunk) * p.n_cols * sizeof(float));
   p.idx_bytes = round256(static_cast<size_t>(ind.n_q) * k * sizeof(int32_t));
   return p;
@@ -290,6 +294,7 @@ dsa_status run_indexer(const dsa_indexer_in& in, const int32_t* rows, int32_t q_
     a.ld_scores = ld_scores;
     a.n_cols = n_cols;
     a.write_masked = write_masked;
+    a.wait_ns = static_cast<uint64_t>(g_wait_ns.load(std::memory_order_relaxed));
     a.status = dev->status;
     DSA_LAUNCH(dsa::launch_indexer_fp8(a, dev->num_sms, pdl, stream));
     return DSA_OK;
@@ -313,15 +318,19 @@ dsa_status run_indexer(const dsa_indexer_in& in, const int32_t* rows, int32_t q_
   return DSA_OK;
 }
 
+// Top-k over n_rows score rows. Row r's position: row_pos[r] when row_pos is
+// set; else, with paged keys (keys != nullptr), that of query pos_base + r;
+// else pos_base + r.
 dsa_status run_topk(const float* scores, int64_t ld_scores, const int32_t* row_pos,
-                    int32_t pos_minus, int32_t pos_base, int32_t n_rows, int32_t k, int32_t* idx, int64_t ld_idx,
-                    bool pdl, DeviceInfo* dev, cudaStream_t stream) {
+                    int32_t pos_base, const dsa::KeySide* keys, int32_t n_rows, int32_t k,
+                    int32_t* idx, int64_t ld_idx, bool pdl, DeviceInfo* dev,
+                    cudaStream_t stream) {
   dsa::TopkArgs a{};
   a.scores = scores;
   a.ld_scores = ld_scores;
   a.row_pos = row_pos;
-  a.pos_minus = pos_minus;
   a.pos_base = pos_base;
+  if (keys != nullptr) a.keys = *keys;
   a.n_rows = n_rows;
   a.k = k;
   a.idx = idx;
@@ -380,26 +389,27 @@ dsa_status run_attn(const dsa_attn_in& in, const int32_t* idx, int64_t ld_idx, i
   return DSA_OK;
 }
 
-// Indexer -> top-k over bounded blocks of query rows (prefill) or all rows at
-// once (paged decode: one row per sequence), scores living only in `scores`.
+// Indexer -> top-k over bounded blocks of `chunk` query rows, the scores of
+// one block living only in `scores` (chunk x n_cols floats). Prefill block
+// rows see keys 0..off+q0+rows-1; paged rows see their sequence's pages.
 dsa_status run_select(const dsa_indexer_in& ind, int32_t k, int32_t* idx, int64_t ld_idx,
-                      float* scores, const ForwardPlan& p, DeviceInfo* dev,
+                      float* scores, int32_t n_cols, int32_t chunk, DeviceInfo* dev,
                       cudaStream_t stream) {
   const int32_t n_q = ind.n_q;
-  if (ind.kv.kind == DSA_KV_PAGED) {
-    DSA_TRY(run_indexer(ind, nullptr, 0, n_q, scores, p.n_cols, p.n_cols, 0, false, dev,
-                        stream));
-    // query b sits at position ctx_lens[b] - 1
-    return run_topk(scores, p.n_cols, ind.kv.ctx_lens, 1, 0, n_q, k, idx, ld_idx, true, dev,
-                    stream);
-  }
-  const int32_t off = ind.n_keys - n_q;  // position of query 0
-  for (int32_t q0 = 0; q0 < n_q; q0 += p.chunk) {
-    const int32_t rows = n_q - q0 < p.chunk ? n_q - q0 : p.chunk;
-    const int32_t cols = off + q0 + rows;  // keys any query of the block sees
+  const bool paged = ind.kv.kind == DSA_KV_PAGED;
+  const int32_t off = paged ? 0 : ind.n_keys - n_q;  // position of query 0 (contiguous)
+  for (int32_t q0 = 0; q0 < n_q; q0 += chunk) {
+    const int32_t rows = n_q - q0 < chunk ? n_q - q0 : chunk;
+    int32_t* out = idx + static_cast<int64_t>(q0) * ld_idx;
+    const int32_t cols = paged ? n_cols : off + q0 + rows;  // keys any row of the block sees
     DSA_TRY(run_indexer(ind, nullptr, q0, rows, scores, cols, cols, 0, q0 > 0, dev, stream));
-    DSA_TRY(run_topk(scores, cols, nullptr, 0, off + q0, rows, k,
-                     idx + static_cast<int64_t>(q0) * ld_idx, ld_idx, true, dev, stream));
+    if (paged) {  // row r is query q0 + r at its own position in its sequence
+      const dsa::KeySide ks = key_side(ind.kv, n_q, ind.n_keys);
+      DSA_TRY(run_topk(scores, cols, nullptr, q0, &ks, rows, k, out, ld_idx, true, dev, stream));
+    } else {
+      DSA_TRY(run_topk(scores, cols, nullptr, off + q0, nullptr, rows, k, out, ld_idx, true, dev,
+                       stream));
+    }
   }
   return DSA_OK;
 }
@@ -434,7 +444,7 @@ DSA_API dsa_status dsa_topk(const float* scores, int64_t ld_scores, const int32_
   if (k < 1 || k > kKMax || ld_idx < k) return DSA_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   DSA_TRY(device_info(&dev));
-  return run_topk(scores, ld_scores, row_pos, 0, 0, n_rows, k, idx, ld_idx, false, dev,
+  return run_topk(scores, ld_scores, row_pos, 0, nullptr, n_rows, k, idx, ld_idx, false, dev,
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -489,7 +499,12 @@ DSA_API dsa_status dsa_forward(const dsa_indexer_in* indexer, const dsa_attn_in*
   const bool paged = indexer->kv.kind == DSA_KV_PAGED;
   if (!paged && indexer->n_keys != attn->n_keys) return DSA_ERR_INVALID_ARG;
   if (paged && (indexer->kv.block_table != attn->kv_layout.block_table ||
-                indexer->kv.ctx_lens != attn->kv_layout.ctx_lens))
+                indexer->kv.ld_block_table != attn->kv_layout.ld_block_table ||
+                indexer->kv.max_pages != attn->kv_layout.max_pages ||
+                indexer->kv.ctx_lens != attn->kv_layout.ctx_lens ||
+                indexer->kv.q_seq != attn->kv_layout.q_seq ||
+                indexer->kv.q_pos != attn->kv_layout.q_pos ||
+                indexer->kv.n_seq != attn->kv_layout.n_seq))
     return DSA_ERR_INVALID_ARG;
   const bool fp8 = indexer->dtype == DSA_E4M3 && attn->dtype == DSA_BF16;
   const bool f32 = indexer->dtype == DSA_F32 && attn->dtype == DSA_F32;
@@ -504,7 +519,8 @@ DSA_API dsa_status dsa_forward(const dsa_indexer_in* indexer, const dsa_attn_in*
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   int32_t* idx = idx_out ? idx_out
                          : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + p.scores_bytes);
-  DSA_TRY(run_select(*indexer, k, idx, k, static_cast<float*>(ws), p, dev, stream));
+  DSA_TRY(run_select(*indexer, k, idx, k, static_cast<float*>(ws), p.n_cols, p.chunk, dev,
+                     stream));
   return run_attn(*attn, idx, k, k, out, lse, dev, stream);
 }
 
@@ -517,11 +533,16 @@ DSA_API dsa_status dsa_select(const dsa_indexer_in* indexer, int32_t k, int32_t*
     return DSA_ERR_WORKSPACE_TOO_SMALL;
   DeviceInfo* dev = nullptr;
   DSA_TRY(device_info(&dev));
-  return run_select(*indexer, k, idx, ld_idx, static_cast<float*>(ws), p, dev,
+  return run_select(*indexer, k, idx, ld_idx, static_cast<float*>(ws), p.n_cols, p.chunk, dev,
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 DSA_API int64_t dsa_launch_counter(void) { return g_launches.load(); }
+
+DSA_API dsa_status dsa_set_wait_limit_ns(int64_t ns) {
+  g_wait_ns.store(ns > 0 ? ns : kDefaultWaitNs, std::memory_order_relaxed);
+  return DSA_OK;
+}
 
 DSA_API dsa_status dsa_check_status(dsa_stream_t stream) {
   DeviceInfo* dev = nullptr;
@@ -551,7 +572,7 @@ DSA_API const char* dsa_status_string(dsa_status s) {
 
 DSA_API int32_t dsa_last_cuda_error(void) { return t_last_cuda_error; }
 
-DSA_API int32_t dsa_version(void) { return 100; }
+DSA_API int32_t dsa_version(void) { return 200; }
 
 }  // extern "C"
 
@@ -611,30 +632,11 @@ extern "C" DSA_API dsa_status dsa_select_noalloc(const dsa_indexer_in* indexer, 
   DSA_TRY(device_info(&dev));
   float* scratch = nullptr;
   DSA_TRY(noalloc_scratch(&scratch));
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  const int32_t n_q = indexer->n_q;
   int64_t block = cap / n_cols;            // query rows whose scores fit at once
   if (block >= 4) block -= block % 4;
-  if (block > n_q) block = n_q;
-  // Every score the top-k reads (columns 0..pos of each row of the block) is
+  if (block > indexer->n_q) block = indexer->n_q;
+  // Every score the top-k reads (columns 0..pos of each row of a block) is
   // written by the indexer launch just before it, so nothing needs clearing.
-  for (int32_t q0 = 0; q0 < n_q; q0 += static_cast<int32_t>(block)) {
-    const int32_t rows = static_cast<int32_t>(n_q - q0 < block ? n_q - q0 : block);
-    int32_t* out = idx + static_cast<int64_t>(q0) * ld_idx;
-    if (paged) {
-      const int32_t cols = static_cast<int32_t>(n_cols);
-      DSA_TRY(run_indexer(*indexer, nullptr, q0, rows, scratch, cols, cols, 0, q0 > 0, dev,
-                          stream));
-      DSA_TRY(run_topk(scratch, cols, indexer->kv.ctx_lens + q0, 1, 0, rows, k, out, ld_idx,
-                       true, dev, stream));
-    } else {
-      const int32_t off = indexer->n_keys - n_q;
-      const int32_t cols = off + q0 + rows;
-      DSA_TRY(run_indexer(*indexer, nullptr, q0, rows, scratch, cols, cols, 0, q0 > 0, dev,
-                          stream));
-      DSA_TRY(run_topk(scratch, cols, nullptr, 0, off + q0, rows, k, out, ld_idx, true, dev,
-                       stream));
-    }
-  }
-  return DSA_OK;
+  return run_select(*indexer, k, idx, ld_idx, scratch, static_cast<int32_t>(n_cols),
+                    static_cast<int32_t>(block), dev, reinterpret_cast<cudaStream_t>(stream_));
 }

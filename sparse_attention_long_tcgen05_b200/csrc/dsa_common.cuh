@@ -25,9 +25,12 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
-// Upper bound of any single wait inside a kernel. Legitimate waits in these
-// kernels last microseconds; one that reaches this bound reports
-// DSA_ERR_TIMEOUT and the waiting role gives up, so a kernel never hangs.
+// Default upper bound of any single wait inside a kernel. Legitimate waits in
+// these kernels last microseconds; one that reaches this bound reports
+// DSA_ERR_TIMEOUT and the waiting role gives up, so a kernel never hangs. The
+// indexer takes its pipeline bound from its launch arguments (this value
+// unless the caller set another); every kernel drains what it has in flight
+// with this bound before it exits.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
 
 // Time a waiting thread may be suspended inside one try_wait before it polls
@@ -65,27 +68,33 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity,
+                                              uint32_t hint_ns = kSuspendHintNs) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
 
 // Waits for the phase with the given parity to complete. Returns false (and
-// records DSA_ERR_TIMEOUT) if that does not happen within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+// records DSA_ERR_TIMEOUT) if that does not happen within limit_ns; a single
+// suspension inside the wait never outlasts the limit either.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+  const uint32_t hint = limit_ns < kSuspendHintNs
+                            ? (limit_ns > 0 ? static_cast<uint32_t>(limit_ns) : 1u)
+                            : kSuspendHintNs;
+  if (mbar_try_wait(a, parity, hint)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
-    if (mbar_try_wait(a, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (mbar_try_wait(a, parity, hint)) return true;
+    if (global_ns() - t0 > limit_ns) {
       report(status, DSA_ERR_TIMEOUT);
       return false;
     }
@@ -122,8 +131,9 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
 // Warp-uniform forms: every lane waits (and acquires) itself, and the result
 // is agreed on by the whole warp, so warp-collective instructions that follow
 // never run with diverged lanes even if a wait times out in some lanes only.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, status));
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, limit_ns));
 }
 
 __device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t* bar, uint32_t parity,

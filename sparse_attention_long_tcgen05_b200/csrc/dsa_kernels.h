@@ -22,11 +22,14 @@ struct KeySide {
   int32_t paged;               // 0 contiguous, 1 paged (64-token pages)
   int32_t n_q;                 // queries in the problem
   int32_t n_keys;              // contiguous: key rows
-  const int32_t* block_table;  // paged
+  const int32_t* block_table;  // paged: [n_seq, ld_block_table]
   int64_t ld_block_table;
   int32_t max_pages;
   int32_t num_pages;
-  const int32_t* ctx_lens;     // paged
+  const int32_t* ctx_lens;     // paged: [n_seq]
+  const int32_t* q_seq;        // paged, nullable: sequence of each query (else query i -> i)
+  const int32_t* q_pos;        // paged, nullable: position of each query (else ctx - 1)
+  int32_t n_seq;               // paged: sequences
 };
 
 // ---------------------------------------------------------------- indexer
@@ -45,6 +48,7 @@ struct IndexerFp8Args {
   int64_t ld_scores;
   int32_t n_cols;
   int32_t write_masked;  // also write -inf for tiles wholly past every query
+  uint64_t wait_ns;      // bound of each pipeline wait (mbarrier) before giving up
   int* status;
 };
 
@@ -77,9 +81,11 @@ cudaError_t launch_indexer_f32(const IndexerF32Args& a, cudaStream_t stream);
 struct TopkArgs {
   const float* scores;
   int64_t ld_scores;
-  const int32_t* row_pos;  // pos = row_pos[r] - pos_minus, or pos_base + r when null
-  int32_t pos_minus;
+  // position of row r: row_pos[r] when row_pos is set; else, for paged keys,
+  // that of query pos_base + r (paged_query); else pos_base + r
+  const int32_t* row_pos;
   int32_t pos_base;
+  KeySide keys;
   int32_t n_rows;
   int32_t k;
   int32_t* idx;
@@ -128,9 +134,25 @@ struct AttnF32Args {
 
 cudaError_t launch_attn_f32(const AttnF32Args& a, cudaStream_t stream);
 
-// Position of query i (shared host/device definition of the ABI rule).
-__host__ __device__ __forceinline__ int32_t query_pos(const KeySide& ks, int32_t qi) {
-  return ks.paged ? ks.ctx_lens[qi] - 1 : ks.n_keys - ks.n_q + qi;
+// Sequence and position of paged query qi (the rule of the ABI's PAGED
+// layout): the sequence is q_seq[qi] (qi when q_seq is null), whose ctx_lens
+// cached tokens include the query's own; the position is q_pos[qi] (ctx - 1
+// when q_pos is null). Returns false -- with seq 0 and pos -1 -- when the
+// sequence, its length or the position is out of range.
+__device__ __forceinline__ bool paged_query(const KeySide& ks, int32_t qi, int32_t& seq,
+                                            int32_t& pos) {
+  seq = ks.q_seq ? ks.q_seq[qi] : qi;
+  pos = -1;
+  if (seq < 0 || seq >= ks.n_seq) {
+    seq = 0;
+    return false;
+  }
+  const int32_t ctx = ks.ctx_lens[seq];
+  if (ctx < 1 || ctx > ks.max_pages * 64) return false;
+  const int32_t p = ks.q_pos ? ks.q_pos[qi] : ctx - 1;
+  if (p < 0 || p >= ctx) return false;
+  pos = p;
+  return true;
 }
 
 }  // namespace dsa

@@ -67,6 +67,7 @@ struct __align__(1024) Smem {
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t acc_full[2], acc_empty[2];
+  uint64_t mma_drain;                // the MMA issuer's own MMAs have all completed
   uint32_t tmem_base;
 };
 
@@ -74,6 +75,7 @@ struct Unit {
   int ng;             // query rows in the group
   int row0;           // first row index
   int qi[kMaxG];      // query indices
+  int seq0;           // paged: block-table row (sequence) of the group's query
   int pos[kMaxG];     // their positions (-1: invalid row, fully masked)
   int max_pos;
   int t0, t1;         // key-tile range of the unit
@@ -88,6 +90,7 @@ __device__ __forceinline__ Unit get_unit(const IndexerFp8Args& a, int G, int n_c
   U.row0 = g * G;
   U.ng = min(G, a.qr.n_rows - U.row0);
   U.max_pos = -1;
+  U.seq0 = 0;
 #pragma unroll
   for (int i = 0; i < kMaxG; ++i) {
     U.qi[i] = 0;
@@ -100,12 +103,11 @@ __device__ __forceinline__ Unit get_unit(const IndexerFp8Args& a, int G, int n_c
         if (report_errors) report(a.status, DSA_ERR_DEVICE_BOUNDS);
         qi = 0;
       } else if (a.keys.paged) {
-        const int ctx = a.keys.ctx_lens[qi];
-        if (ctx < 1 || ctx > a.keys.max_pages * 64) {
-          if (report_errors) report(a.status, DSA_ERR_DEVICE_BOUNDS);
-        } else {
-          pos = ctx - 1;
-        }
+        // one query per group in paged mode (G = 1)
+        int seq;
+        if (!paged_query(a.keys, qi, seq, pos) && report_errors)
+          report(a.status, DSA_ERR_DEVICE_BOUNDS);
+        U.seq0 = seq;
       } else {
         pos = a.keys.n_keys - a.keys.n_q + qi;
       }
@@ -121,9 +123,10 @@ __device__ __forceinline__ Unit get_unit(const IndexerFp8Args& a, int G, int n_c
   return U;
 }
 
-// Page id of logical page p of query qi, checked; 0 when out of range.
-__device__ __forceinline__ int page_of(const IndexerFp8Args& a, int qi, int p, bool report_errors) {
-  int page = a.keys.block_table[static_cast<int64_t>(qi) * a.keys.ld_block_table + p];
+// Page id of logical page p of sequence seq, checked; 0 when out of range.
+__device__ __forceinline__ int page_of(const IndexerFp8Args& a, int seq, int p,
+                                       bool report_errors) {
+  int page = a.keys.block_table[static_cast<int64_t>(seq) * a.keys.ld_block_table + p];
   if (page < 0 || page >= a.keys.num_pages) {
     if (report_errors) report(a.status, DSA_ERR_DEVICE_BOUNDS);
     page = 0;
@@ -158,6 +161,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
       // reads the stage's key scales (half of them with one query per group)
       mbar_init(&S.k_empty[i], 1 + (G == 1 ? kEpiThreads / 2 : kEpiThreads));
     }
+    mbar_init(&S.mma_drain, 1);
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -182,26 +186,33 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
     int it = 0, ks = 0;
     uint32_t kph = 0;
     bool ok = true;
+    // loads issued per buffer / stage, so the drain below knows which phases
+    // to wait for
+    uint32_t q_fills[2] = {0u, 0u};
+    uint32_t k_fills[kStages];
+#pragma unroll
+    for (int i = 0; i < kStages; ++i) k_fills[i] = 0u;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
       const Unit U = get_unit(a, G, n_chunks, n_tiles, tpu, u, first && lane == 0);
       const int qb = it & 1;
       const uint32_t qph = (it >> 1) & 1;
       if (first) {
-        if (!mbar_wait_warp(&S.q_empty[qb], qph ^ 1, a.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&S.q_empty[qb], qph ^ 1, a.status, a.wait_ns)) { ok = false; break; }
         if (lane == 0) {
           mbar_arrive_expect_tx(&S.q_full[qb], U.ng * kQBytes);
           for (int i = 0; i < U.ng; ++i)
             tma_load_3d(S.q[qb] + i * kQBytes, &a.map_q, 0, 0, U.qi[i], &S.q_full[qb]);
         }
+        ++q_fills[qb];
       }
       int pg = -1;     // page of logical page 2 t0 + lane, if it holds a key <= max_pos
       if (a.keys.paged) {
         const int p = 2 * U.t0 + lane;
         if (lane < 2 * (U.t_end - U.t0) && p * 64 <= U.max_pos)
-          pg = page_of(a, U.qi[0], p, first);
+          pg = page_of(a, U.seq0, p, first);
       }
       for (int t = U.t0; t < U.t_end; ++t) {
-        if (!mbar_wait_warp(&S.k_empty[ks], kph ^ 1, a.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&S.k_empty[ks], kph ^ 1, a.status, a.wait_ns)) { ok = false; break; }
         const int i0 = 2 * (t - U.t0);
         const int pg0 = __shfl_sync(0xffffffffu, pg, i0 & 31);
         const int pg1 = __shfl_sync(0xffffffffu, pg, (i0 + 1) & 31);
@@ -219,9 +230,24 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
             tma_load_1d(S.sk[ks] + 64, &a.map_sk, pg1u * 64, &S.k_full[ks]);
           }
         }
+#pragma unroll
+        for (int i = 0; i < kStages; ++i) k_fills[i] += i == ks ? 1u : 0u;
         if (++ks == kStages) { ks = 0; kph ^= 1; }
       }
     }
+    // Drain: after a give-up the consumers may never have waited for the last
+    // loads; wait (with the default bound) until every load this warp issued
+    // has landed, so no copy is still writing shared memory when the CTA
+    // exits. On the normal path each of these phases completed long ago.
+    if (lane == 0) {
+      if (first)
+        for (int b = 0; b < 2; ++b)
+          if (q_fills[b]) mbar_wait(&S.q_full[b], (q_fills[b] - 1u) & 1u, a.status);
+#pragma unroll
+      for (int i = 0; i < kStages; ++i)
+        if (k_fills[i]) mbar_wait(&S.k_full[i], (k_fills[i] - 1u) & 1u, a.status);
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -233,7 +259,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
         const Unit U = get_unit(a, G, n_chunks, n_tiles, tpu, u, false);
         const int qb = it & 1;
         const uint32_t qph = (it >> 1) & 1;
-        if (!mbar_wait(&S.q_full[qb], qph, a.status)) break;
+        if (!mbar_wait(&S.q_full[qb], qph, a.status, a.wait_ns)) break;
         tc_fence_after();
         const uint64_t bdesc = sw128_desc(smem_u32(S.q[qb]), 16, 1024);
         if (G == 1) {
@@ -241,11 +267,11 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           // 128-column accumulator
           for (int t = U.t0; t < U.t_end && ok; t += 2) {
             const int nt = min(2, U.t_end - t);
-            if (!mbar_wait(&S.acc_empty[ab], aph ^ 1, a.status)) { ok = false; break; }
+            if (!mbar_wait(&S.acc_empty[ab], aph ^ 1, a.status, a.wait_ns)) { ok = false; break; }
             for (int h = 0; h < nt && ok; ++h) {
               const int kss = ks + h < kStages ? ks + h : ks + h - kStages;
               const uint32_t kp = ks + h < kStages ? kph : kph ^ 1u;
-              if (!mbar_wait(&S.k_full[kss], kp, a.status)) ok = false;
+              if (!mbar_wait(&S.k_full[kss], kp, a.status, a.wait_ns)) ok = false;
             }
             if (!ok) break;
             tc_fence_after();
@@ -268,7 +294,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
         }
         for (int t = U.t0; t < U.t_end; ++t) {
           if (!mbar_wait(&S.k_full[ks], kph, a.status) ||
-              !mbar_wait(&S.acc_empty[ab], aph ^ 1, a.status)) { ok = false; break; }
+              !mbar_wait(&S.acc_empty[ab], aph ^ 1, a.status, a.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = sw128_desc(smem_u32(S.k[ks]), 16, 1024);
           const uint32_t d = tmem_base + static_cast<uint32_t>(ab * N);
@@ -282,7 +308,12 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
         }
         mma_commit(&S.q_empty[qb]);
       }
+      // Drain: the MMAs issued so far (possibly none) complete before TMEM is
+      // freed and before the operands' shared memory goes away.
+      mma_commit(&S.mma_drain);
+      mbar_wait(&S.mma_drain, 0, a.status);
     }
+    __syncwarp();
   } else if (warp >= 2 && warp < kPageWarp) {
     // ------------------------------------------------------------ epilogue
     const int sub = warp & 3;              // TMEM sub-partition of this warp
@@ -320,11 +351,11 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           if (mine) {
             const int kss = ks + half < kStages ? ks + half : ks + half - kStages;
             const uint32_t kp = ks + half < kStages ? kph : kph ^ 1u;
-            if (!mbar_wait_warp(&S.k_full[kss], kp, a.status)) { ok = false; break; }
+            if (!mbar_wait_warp(&S.k_full[kss], kp, a.status, a.wait_ns)) { ok = false; break; }
             sk = S.sk[kss][sub * 32 + lane];
             mbar_arrive(&S.k_empty[kss]);
           }
-          if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status)) { ok = false; break; }
+          if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status, a.wait_ns)) { ok = false; break; }
           tc_fence_after();
           if (mine) {
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) +
@@ -364,11 +395,11 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           continue;
         }
         // this tile's key scale (the stage also holds the key codes)
-        if (!mbar_wait_warp(&S.k_full[ks], kph, a.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&S.k_full[ks], kph, a.status, a.wait_ns)) { ok = false; break; }
         const float sk = S.sk[ks][sub * 32 + lane];
         mbar_arrive(&S.k_empty[ks]);
         if (++ks == kStages) { ks = 0; kph ^= 1; }
-        if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status, a.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) +
                                static_cast<uint32_t>(ab * N + g0 * kHeads);

@@ -227,12 +227,10 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
   const int col0 = 256 * static_cast<int>(rank);
   const int qi = blockIdx.x >> 1;
 
-  int pos;
+  int pos, seq = 0;
   bool q_ok = true;
   if (a.keys.paged) {
-    const int ctx = a.keys.ctx_lens[qi];
-    q_ok = ctx >= 1 && ctx <= a.keys.max_pages * 64;
-    pos = q_ok ? ctx - 1 : -1;
+    q_ok = paged_query(a.keys, qi, seq, pos);
   } else {
     pos = a.keys.n_keys - a.keys.n_q + qi;
   }
@@ -302,7 +300,7 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
       for (int i = 0; i < 4; ++i)
         pg[i] = (a.keys.paged && e[i] >= 0)
                     ? __ldg(a.keys.block_table +
-                            static_cast<int64_t>(qi) * a.keys.ld_block_table + (e[i] >> 6))
+                            static_cast<int64_t>(seq) * a.keys.ld_block_table + (e[i] >> 6))
                     : 0;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {

@@ -221,7 +221,15 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
   int32_t* out = a.idx + static_cast<int64_t>(r) * a.ld_idx;
   griddep_launch_dependents();
   griddep_wait();   // the score rows come from the kernel before this one
-  const int pos = a.row_pos ? a.row_pos[r] - a.pos_minus : a.pos_base + r;
+  int pos;
+  if (a.row_pos) {
+    pos = a.row_pos[r];
+  } else if (a.keys.paged) {
+    int seq;
+    paged_query(a.keys, a.pos_base + r, seq, pos);   // -1 when out of range
+  } else {
+    pos = a.pos_base + r;
+  }
   if (pos < 0 || pos >= a.ld_scores) {
     if (tid == 0) report(a.status, DSA_ERR_DEVICE_BOUNDS);
     for (int j = tid; j < a.k; j += kThreads) out[j] = -1;

@@ -33,7 +33,8 @@ DSA_OP_SELECT = 4
 
 EXPORTED = ["dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_fwd", "dsa_select", "dsa_forward",
             "dsa_workspace_size", "dsa_check_status", "dsa_status_string",
-            "dsa_last_cuda_error", "dsa_launch_counter", "dsa_version", "dsa_select_noalloc"]
+            "dsa_last_cuda_error", "dsa_launch_counter", "dsa_version", "dsa_select_noalloc",
+            "dsa_set_wait_limit_ns"]
 
 
 class DsaError(RuntimeError):
@@ -46,7 +47,8 @@ class KvLayout(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("page_size", ctypes.c_int32),
                 ("block_table", ctypes.c_void_p), ("ld_block_table", ctypes.c_int64),
                 ("max_pages", ctypes.c_int32), ("num_pages", ctypes.c_int32),
-                ("ctx_lens", ctypes.c_void_p)]
+                ("ctx_lens", ctypes.c_void_p), ("q_seq", ctypes.c_void_p),
+                ("q_pos", ctypes.c_void_p), ("n_seq", ctypes.c_int32)]
 
 
 class IndexerIn(ctypes.Structure):
@@ -80,6 +82,7 @@ def _load():
         "dsa_select": [ctypes.POINTER(IndexerIn), I32, P, I64, P, SZ, P],
         "dsa_forward": [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), I32, P, P, P, P, SZ, P],
         "dsa_launch_counter": [],
+        "dsa_set_wait_limit_ns": [I64],
         "dsa_select_noalloc": [ctypes.POINTER(IndexerIn), I32, P, I64, P],
         "dsa_workspace_size": [I32, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), I32, I32,
                                I32, ctypes.POINTER(SZ)],
@@ -129,9 +132,17 @@ class _Keep:
         self.tensors = tensors
 
 
-def paged_layout(block_table: torch.Tensor, ctx_lens: torch.Tensor, num_pages: int) -> KvLayout:
+def paged_layout(block_table: torch.Tensor, ctx_lens: torch.Tensor, num_pages: int,
+                 q_seq: Optional[torch.Tensor] = None,
+                 q_pos: Optional[torch.Tensor] = None) -> KvLayout:
+    """PAGED key side: block_table [n_seq, max_pages] and ctx_lens [n_seq]
+    int32; optional q_seq / q_pos [n_q] int32 (sequence and position of each
+    query; by default query b is the newest token of sequence b). The caller
+    keeps the tensors alive while the layout is in use."""
     return KvLayout(DSA_KV_PAGED, 64, block_table.data_ptr(), block_table.stride(0),
-                    block_table.shape[1], num_pages, ctx_lens.data_ptr())
+                    block_table.shape[1], num_pages, ctx_lens.data_ptr(),
+                    q_seq.data_ptr() if q_seq is not None else None,
+                    q_pos.data_ptr() if q_pos is not None else None, ctx_lens.shape[0])
 
 
 def indexer_in(q, k, w, q_scale=None, k_scale=None, n_keys=None, kv: Optional[KvLayout] = None):
@@ -212,6 +223,11 @@ def dsa_select_noalloc(ind: _Keep, k: int, idx: torch.Tensor, stream=None):
     Calls on one device must not overlap (they share that scratch)."""
     _check(LIB.dsa_select_noalloc(ctypes.byref(ind.struct), k, _ptr(idx), idx.stride(0),
                                   _stream(stream)), "dsa_select_noalloc")
+
+
+def dsa_set_wait_limit_ns(ns: int):
+    """Bound of the indexer kernel's pipeline waits (ns <= 0: the 1 s default)."""
+    _check(LIB.dsa_set_wait_limit_ns(int(ns)), "dsa_set_wait_limit_ns")
 
 
 def dsa_launch_counter() -> int:

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_status_strings_and_version(lib):
     assert lib.status_string(0) == "ok"
     assert "range" in lib.status_string(lib.DSA_ERR_DEVICE_BOUNDS)
-    assert lib.LIB.dsa_version() >= 100
+    assert lib.LIB.dsa_version() >= 200
 
 
 def test_workspace_size_host_logic(lib):
@@ -80,8 +80,10 @@ def test_struct_layout_matches_c(lib):
 #include <stddef.h>
 #include "dsa.h"
 int main(void) {
-  printf("%zu %zu %zu %zu\n", sizeof(dsa_kv_layout), offsetof(dsa_kv_layout, block_table),
-         offsetof(dsa_kv_layout, ld_block_table), offsetof(dsa_kv_layout, ctx_lens));
+  printf("%zu %zu %zu %zu %zu %zu %zu\n", sizeof(dsa_kv_layout),
+         offsetof(dsa_kv_layout, block_table), offsetof(dsa_kv_layout, ld_block_table),
+         offsetof(dsa_kv_layout, ctx_lens), offsetof(dsa_kv_layout, q_seq),
+         offsetof(dsa_kv_layout, q_pos), offsetof(dsa_kv_layout, n_seq));
   printf("%zu %zu %zu %zu %zu %zu\n", sizeof(dsa_indexer_in), offsetof(dsa_indexer_in, q),
          offsetof(dsa_indexer_in, q_scale), offsetof(dsa_indexer_in, w),
          offsetof(dsa_indexer_in, ld_w), offsetof(dsa_indexer_in, kv));
@@ -99,6 +101,7 @@ int main(void) {
     got = [int(x) for x in got]
     K, I, A = lib.KvLayout, lib.IndexerIn, lib.AttnIn
     want = [ctypes.sizeof(K), K.block_table.offset, K.ld_block_table.offset, K.ctx_lens.offset,
+            K.q_seq.offset, K.q_pos.offset, K.n_seq.offset,
             ctypes.sizeof(I), I.q.offset, I.q_scale.offset, I.w.offset, I.ld_w.offset,
             I.kv.offset,
             ctypes.sizeof(A), A.scale.offset, A.q.offset, A.v.offset, A.kv_layout.offset]

@@ -2,10 +2,10 @@
 kernels, called through the C ABI) against the oracle.
 
 Small cases cover every row and end in ragged tails (key tiles of 128, query
-groups of 4, key blocks of 64); the L=4096 workload is checked on every row for
-the indexer mask and the top-k, and on sampled rows for values; the 32K and
-128K workloads on sampled rows in the same launch configuration the benchmark
-times (dsa_forward)."""
+groups of 4, key blocks of 64); the L=4096 workload is checked on every row
+(indexer values and mask, the selection, the attention output); the 32K and
+128K workloads on the same seeded sample of 512 query rows, in the launch
+configuration the benchmark times (dsa_forward)."""
 import dataclasses
 import os
 
@@ -264,30 +264,41 @@ def _forward(dsa, T, inp):
     return ind, att, idx, out, lse
 
 
-def _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, rows):
+def _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, rows, chunk=128):
+    """Element-wise parity of the fused forward on the given query rows,
+    checked in chunks of rows so the host copies stay bounded at 128K:
+    indexer values against the oracle, the fused selection against the
+    oracle's top-k of the same float32 scores (bit-exact), and the attention
+    output against the oracle's attention over that selection."""
     wl = inp.wl
     L, k = wl.L, wl.k
-    # indexer values on the sampled rows
-    sc = _scores(dsa, ind, rows, L)
-    qi, ki, w, q = T.oracle_prefill_inputs(inp, rows)
-    ref_scores = T.oracle_scores(qi, ki, w, rows, L)
-    T.assert_indexer_close(sc.cpu().numpy(), ref_scores)
-    # the fused selection equals top-k of the standalone scores, bit for bit,
-    # and equals the oracle's top-k of those same scores
-    r = torch.tensor(rows, device="cuda")
-    g_idx = idx[r].cpu().numpy()
-    ref_idx = T.topk_oracle_on(sc.double().cpu().numpy(), np.array(rows), k)
-    assert np.array_equal(g_idx, ref_idx)
-    # attention on the sampled rows with those indices
-    kv_sub, idx_local = T.gather_kv_rows(inp.kv, g_idx)
-    o_ref, l_ref = O.sparse_mqa(q, kv_sub, None, idx_local, list(range(len(rows))), wl.scale,
-                                512)
-    T.assert_attention_close(out[r].float().cpu().numpy(), lse[r].cpu().numpy(), o_ref, l_ref)
-    # diagnostic: overlap with the oracle's own selection (its own scores)
-    own = T.topk_oracle_on(ref_scores, np.array(rows), k)
-    overlap = np.mean([len(set(a[a >= 0]) & set(b[b >= 0])) / max(1, (b >= 0).sum())
-                       for a, b in zip(g_idx, own)])
-    assert overlap > 0.95, overlap
+    k_deq = T.oracle_key_side(inp)
+    overlaps = []
+    for c0 in range(0, len(rows), chunk):
+        part = list(rows[c0:c0 + chunk])
+        # indexer values on these rows
+        sc = _scores(dsa, ind, part, L)
+        qi, w, q = T.oracle_query_side(inp, part)
+        ref_scores = T.oracle_scores(qi, k_deq, w, part, L)
+        g_sc = sc.cpu().numpy()
+        T.assert_indexer_close(g_sc, ref_scores)
+        # the fused selection equals top-k of the standalone scores, bit for
+        # bit, and equals the oracle's top-k of those same scores
+        r = torch.tensor(part, device="cuda")
+        g_idx = idx[r].cpu().numpy()
+        ref_idx = T.topk_oracle_on(g_sc.astype(np.float64), np.array(part), k)
+        assert np.array_equal(g_idx, ref_idx)
+        # attention on these rows with those indices
+        kv_sub, idx_local = T.gather_kv_rows(inp.kv, g_idx)
+        o_ref, l_ref = O.sparse_mqa(q, kv_sub, None, idx_local, list(range(len(part))),
+                                    wl.scale, 512)
+        T.assert_attention_close(out[r].float().cpu().numpy(), lse[r].cpu().numpy(), o_ref,
+                                 l_ref)
+        # diagnostic: overlap with the oracle's own selection (its own scores)
+        own = T.topk_oracle_on(ref_scores, np.array(part), k)
+        overlaps += [len(set(a[a >= 0]) & set(b[b >= 0])) / max(1, (b >= 0).sum())
+                     for a, b in zip(g_idx, own)]
+    assert np.mean(overlaps) > 0.95, np.mean(overlaps)
 
 
 def test_forward_L4096(libs):
@@ -310,7 +321,8 @@ def test_forward_L4096(libs):
     cnt = (ih >= 0).sum(1)
     assert np.array_equal(cnt, np.minimum(k, np.arange(L) + 1))
     assert np.all(ih.max(1) <= np.arange(L))
-    _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, sample_rows(L, 64, seed=1))
+    # every row: indexer values, selection and attention against the oracle
+    _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, list(range(L)), chunk=512)
 
 
 @pytest.mark.parametrize("L", [5000, 16384])
@@ -336,7 +348,7 @@ def test_forward_L32768_needles(libs):
     dsa, T = libs
     inp = make_prefill(WORKLOADS[2], device="cuda", seed=0)
     ind, att, idx, out, lse = _forward(dsa, T, inp)
-    rows = sample_rows(inp.wl.L, 48, seed=1)
+    rows = sample_rows(inp.wl.L, 512, seed=1)
     _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, rows)
     # the planted x3 keys are over-represented in the selections of long rows
     needles = set(inp.needles.cpu().tolist())
@@ -354,8 +366,81 @@ def test_forward_L131072_sampled(libs):
     dsa, T = libs
     inp = make_prefill(WORKLOADS[3], device="cuda", seed=0)
     ind, att, idx, out, lse = _forward(dsa, T, inp)
-    n = int(os.environ.get("DSA_128K_ROWS", "32"))
+    n = int(os.environ.get("DSA_128K_ROWS", "512"))
     rows = sample_rows(inp.wl.L, n, seed=1)
     _check_forward_rows(dsa, T, inp, ind, att, idx, out, lse, rows)
     ih = idx[torch.tensor(rows, device="cuda")].cpu().numpy()
     assert np.array_equal((ih >= 0).sum(1), np.minimum(2048, np.array(rows) + 1))
+
+
+def _suffix_structs(dsa, inp, off):
+    """Structs for the queries off..L-1 of a prefill against all L keys (a
+    chunk of a longer prefill): query i sits at position off + i."""
+    wl = inp.wl
+    ind = dsa.indexer_in(inp.q_idx[off:], inp.k_idx, inp.w[off:], inp.q_scale[off:],
+                         inp.k_scale)
+    att = dsa.attn_in(inp.q[off:], inp.kv, wl.scale, wl.D_V)
+    return ind, att
+
+
+def test_attention_bf16_query_suffix(libs):
+    """Chunked prefill: 300 queries at positions 700..999 attend over their own
+    selections among 1000 keys (entries up to each query's position)."""
+    dsa, T = libs
+    L, off, k = 1000, 700, 512
+    inp = make_prefill(_wl(L, k), device="cuda", seed=21)
+    rng = np.random.default_rng(21)
+    rows = np.arange(off, L)
+    idx_h = T.topk_oracle_on(rng.standard_normal((L - off, L)), rows, k)
+    _, att = _suffix_structs(dsa, inp, off)
+    out = torch.empty(L - off, 128, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(L - off, 128, device="cuda")
+    dsa.dsa_sparse_mqa_fwd(att, torch.from_numpy(idx_h).cuda(), k, out, lse)
+    assert dsa.dsa_check_status() == 0
+    q = inp.q[off:].double().cpu().numpy()
+    kv_sub, idx_local = T.gather_kv_rows(inp.kv, idx_h)
+    o_ref, l_ref = O.sparse_mqa(q, kv_sub, None, idx_local, list(range(L - off)), inp.wl.scale,
+                                512)
+    T.assert_attention_close(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref)
+
+
+@pytest.mark.parametrize("L,off", [(3000, 1700), (9000, 8000)])
+def test_forward_query_suffix_every_row(libs, L, off):
+    """dsa_forward on a chunk of a longer prefill (queries off..L-1 against all
+    L keys; 9000/8000 gives rows with more than k candidates and a suffix that
+    is not a multiple of the 4-query groups): every row's indexer values,
+    selection and attention against the oracle at the query's own position,
+    and the selection equals the same rows of the whole prefill's selection."""
+    dsa, T = libs
+    k = 2048
+    inp = make_prefill(_wl(L, k), device="cuda", seed=22)
+    ind, att = _suffix_structs(dsa, inp, off)
+    n_q = L - off
+    ws = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_FORWARD, ind, att, 0, 0, k))
+    idx = torch.empty(n_q, k, dtype=torch.int32, device="cuda")
+    out = torch.empty(n_q, 128, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(n_q, 128, device="cuda")
+    dsa.dsa_forward(ind, att, k, idx, out, lse, ws)
+    assert dsa.dsa_check_status() == 0
+    # standalone scores of the suffix rows (row r = query r, position off + r)
+    sc = torch.empty(n_q, L, device="cuda")
+    dsa.dsa_indexer_scores(ind, None, n_q, sc, L)
+    assert dsa.dsa_check_status() == 0
+    pos = np.arange(off, L)
+    k_deq = T.oracle_key_side(inp)
+    qi, w, q = T.oracle_query_side(inp, list(pos))
+    ref = T.oracle_scores(qi, k_deq, w, list(pos), L)
+    g_sc = sc.cpu().numpy()
+    T.assert_indexer_close(g_sc, ref)
+    g_idx = idx.cpu().numpy()
+    assert np.array_equal(g_idx, T.topk_oracle_on(g_sc.astype(np.float64), pos, k))
+    kv_sub, idx_local = T.gather_kv_rows(inp.kv, g_idx)
+    o_ref, l_ref = O.sparse_mqa(q, kv_sub, None, idx_local, list(range(n_q)), inp.wl.scale, 512)
+    T.assert_attention_close(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref)
+    # the same rows of the whole prefill select the same keys
+    full_ind, _ = T.prefill_structs(inp)
+    ws2 = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_SELECT, full_ind, None, 0, 0, k))
+    idx_full = torch.empty(L, k, dtype=torch.int32, device="cuda")
+    dsa.dsa_select(full_ind, k, idx_full, ws2)
+    assert dsa.dsa_check_status() == 0
+    assert torch.equal(idx_full[off:], idx)

@@ -58,6 +58,23 @@ def test_noalloc_select_prefill_matches_workspace_form(dsa):
         assert torch.equal(got, ref)
 
 
+def test_noalloc_select_query_suffix_matches_workspace_form(dsa):
+    # the queries are the last 2000 tokens of 6000 keys (a chunk of a longer
+    # prefill): each block's rows see keys 0..4000+q0+rows-1; the scratch holds
+    # 696 rows of 6000 scores, so the 2000 queries run as 3 blocks
+    wl = dataclasses.replace(WORKLOADS[1], L=6000)
+    inp = make_prefill(wl, device="cuda", seed=13)
+    off = 4000
+    ind = dsa.indexer_in(inp.q_idx[off:], inp.k_idx, inp.w[off:], inp.q_scale[off:],
+                         inp.k_scale)
+    ref = _with_workspace(dsa, ind, wl.k, wl.L - off)
+    for _ in range(2):
+        got = torch.full_like(ref, -7)
+        _noalloc(dsa, ind, wl.k, got)
+        assert dsa.dsa_check_status() == 0
+        assert torch.equal(got, ref)
+
+
 def test_noalloc_select_paged_matches_workspace_form(dsa):
     # 2048 pages x 64 = 131072 columns per row: 32 rows per block, 40 sequences
     wl = dataclasses.replace(WORKLOADS[4], ctx_max=131072)
