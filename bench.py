@@ -372,6 +372,10 @@ def run_ours(args, world, rank, local):
     dom = "indexer_fp8_kernel" if ms_idx > ms_attn else "sparse_mqa_bf16_kernel"
     roof = dict(rooflines[dom], kernel=dom)
 
+    curve = None
+    if not args.skip_curve:
+        curve = cost_vs_position(dsa, inp, wl, k, world, peaks)
+
     # ------------------------------------------------------------ e2e (host buffers)
     e2e = None
     if not args.skip_e2e:
@@ -396,7 +400,7 @@ def run_ours(args, world, rank, local):
                    "l2": "inputs larger than L2 (q alone 19.3 GB)",
                    "parallelism": f"replicas x{world} (independent sequences)"},
         "roofline": roof, "rooflines": rooflines, "fp8_peak": fp8, "stages": stages,
-        "cpu_baseline": cpu, "e2e": e2e,
+        "cpu_baseline": cpu, "e2e": e2e, "cost_vs_position": curve,
         "gpu_launches": int(round(per_call * args.steps)),
         "clocks": clk.summary(),
     }
@@ -406,6 +410,41 @@ def run_ours(args, world, rank, local):
         res["decode"] = run_decode(args, world, rank, local, peaks, dsa, make_decode,
                                    WORKLOADS[DECODE_WL])
     return res
+
+
+def cost_vs_position(dsa, inp, wl, k, world, peaks, block=4096, steps=2,
+                     positions=(4096, 8192, 16384, 32768, 65536, 98304, 131072)):
+    """Prefill cost per token position: for each P, the block of `block`
+    queries at positions P-block .. P-1 against keys 0..P-1 (a chunk of the
+    prefill), timed once through dsa_forward (indexer -> top-k -> sparse
+    attention) and once through dsa_dense_mqa_fwd (dense causal attention, the
+    baseline DSA replaces), on the same inputs. ms per block of queries."""
+    out = torch.empty(block, wl.H, wl.D_V, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(block, wl.H, device="cuda")
+    idx = torch.empty(block, k, dtype=torch.int32, device="cuda")
+    pts = []
+    for P in positions:
+        if P > wl.L or P < block:
+            continue
+        off = P - block
+        ind = dsa.indexer_in(inp.q_idx[off:P], inp.k_idx[:P], inp.w[off:P], inp.q_scale[off:P],
+                             inp.k_scale[:P])
+        att = dsa.attn_in(inp.q[off:P], inp.kv[:P], wl.scale, wl.D_V)
+        ws = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_FORWARD, ind, att, 0, 0, k))
+        ms_dsa = timed(lambda: dsa.dsa_forward(ind, att, k, idx, out, lse, ws), steps, 1, world)
+        ms_dense = timed(lambda: dsa.dsa_dense_mqa_fwd(att, out, lse), steps, 1, world)
+        st = dsa.dsa_check_status()
+        if st != 0:
+            raise RuntimeError(f"device status {dsa.status_string(st)}")
+        keys = block * (off + 1) + block * (block - 1) // 2          # sum of (t + 1)
+        dense_tf = 2.0 * wl.H * (wl.D_K + wl.D_V) * keys / (ms_dense * 1e-3) / 1e12
+        pts.append({"position": P, "dsa_ms": ms_dsa, "dense_ms": ms_dense,
+                    "dense_over_dsa": ms_dense / ms_dsa, "dense_bf16_tflops": dense_tf,
+                    "dense_frac_bf16_sustained": dense_tf / peaks["bf16_sustained"]})
+        del ws
+    return {"block_queries": block, "unit": "ms per block of queries", "points": pts,
+            "how": "queries P-block..P-1 against keys 0..P-1 of the 128K inputs; dsa = "
+                   "dsa_forward (indexer, top-k, sparse attention), dense = dsa_dense_mqa_fwd"}
 
 
 def prefill_e2e(dsa, inp, ind, att, ws, idx, out, lse, k, args, world, n_chunks=8):
@@ -638,6 +677,8 @@ def main():
                          "for multi-pass profiling")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-curve", action="store_true",
+                    help="skip the prefill cost-vs-position curve (DSA against dense)")
     ap.add_argument("--skip-fp8-peak", action="store_true",
                     help="do not measure the FP8 GEMM peak (the indexer is then reported "
                          "against 2 x the bf16 peak)")

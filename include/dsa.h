@@ -192,6 +192,20 @@ DSA_API dsa_status dsa_sparse_mqa_fwd(const dsa_attn_in* in, const int32_t* idx,
                                       int32_t k, void* out, float* lse, void* ws,
                                       size_t ws_bytes, dsa_stream_t stream);
 
+/* Dense causal MLA-MQA attention: the baseline that DSA replaces, in which
+ * every query attends to all of its preceding tokens (paperbridge.wiki
+ * summary, section on dense attention; the pages compare DSA's prefill and
+ * decode cost per token position against it: juhe.plus read-through, sparse
+ * training stage; 53ai.com read-through, Figure 3). Query i (position pos, as
+ * in "Positions") attends to keys 0..pos with the same inputs and outputs as
+ * dsa_sparse_mqa_fwd, as if its selection held every key. Results equal
+ * dsa_sparse_mqa_fwd with idx = 0..pos (ascending) bit for bit when pos < k.
+ * BF16: CONTIGUOUS or PAGED; a PAGED query with a page id out of range among
+ * its pages is reported as DSA_ERR_DEVICE_BOUNDS and gets a zero output.
+ * F32: CONTIGUOUS, n_keys <= 4096. No workspace. */
+DSA_API dsa_status dsa_dense_mqa_fwd(const dsa_attn_in* in, void* out, float* lse,
+                                     dsa_stream_t stream);
+
 /* Steps 1-2 fused: the selection alone (indexer -> top-k), streamed over
  * bounded blocks of queries so the n_q x n_keys score matrix never exists.
  * idx: [n_q, ld_idx] int32 (ld_idx >= k), same contents and rules as

@@ -29,6 +29,7 @@ std::atomic<int64_t> g_wait_ns{kDefaultWaitNs};
 constexpr int kMaxDevices = 64;
 constexpr int kKMax = 2048;
 constexpr int kPage = 64;
+constexpr int kDenseF32MaxKeys = 4096;
 
 struct DeviceInfo {
   bool init = false;
@@ -347,15 +348,8 @@ dsa_status run_attn(const dsa_attn_in& in, const int32_t* idx, int64_t ld_idx, i
     dsa::AttnBf16Args a{};
     a.q = static_cast<const __nv_bfloat16*>(in.q);
     a.ld_q = in.ld_q;
-    {
-      const uint64_t rows_kv = ks.paged ? static_cast<uint64_t>(in.kv_layout.num_pages) * kPage
-                                        : static_cast<uint64_t>(in.n_keys);
-      const uint64_t dims[2] = {576, rows_kv};
-      const uint64_t strides[1] = {static_cast<uint64_t>(in.ld_kv) * 2};
-      const uint32_t box[2] = {64, 1};
-      DSA_TRY(make_map(&a.map_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, in.kv, dims, strides,
-                       box, CU_TENSOR_MAP_SWIZZLE_128B));
-    }
+    a.kv = static_cast<const __nv_bfloat16*>(in.kv);
+    a.ld_kv = in.ld_kv;
     a.idx = idx;
     a.ld_idx = ld_idx;
     a.k = k;
@@ -460,6 +454,19 @@ DSA_API dsa_status dsa_sparse_mqa_fwd(const dsa_attn_in* in, const int32_t* idx,
   DeviceInfo* dev = nullptr;
   DSA_TRY(device_info(&dev));
   return run_attn(*in, idx, ld_idx, k, out, lse, dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+DSA_API dsa_status dsa_dense_mqa_fwd(const dsa_attn_in* in, void* out, float* lse,
+                                     dsa_stream_t stream) {
+  DSA_TRY(check_attn(in));
+  if (out == nullptr) return DSA_ERR_INVALID_ARG;
+  if (in->dtype == DSA_BF16 && !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  // the fp32 kernel keeps one probability per key in shared memory
+  if (in->dtype == DSA_F32 && in->n_keys > kDenseF32MaxKeys) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  DSA_TRY(device_info(&dev));
+  return run_attn(*in, nullptr, 0, in->dtype == DSA_F32 ? in->n_keys : 0, out, lse, dev,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 DSA_API dsa_status dsa_workspace_size(int32_t op, const dsa_indexer_in* indexer,

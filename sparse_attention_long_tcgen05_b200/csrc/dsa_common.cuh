@@ -249,6 +249,27 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// ------------------------------------------------------------------ cp.async
+
+// 16 bytes global -> shared, asynchronous, through L2 only (no L1 allocation).
+// Both addresses 16-byte aligned. The data is written by the generic proxy:
+// the issuing thread waits for its group (cp_async_wait_group) and fences
+// (fence_proxy_async_smem) before a tensor-core read may be released to it.
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Waits until at most N of this thread's committed groups are still pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05 / TMEM
 
 // Allocates `ncols` TMEM columns (power of two >= 32); the address is written

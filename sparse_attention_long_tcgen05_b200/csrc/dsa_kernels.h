@@ -99,7 +99,8 @@ cudaError_t launch_topk(const TopkArgs& a, bool pdl, cudaStream_t stream);
 // ---------------------------------------------------------------- attention
 
 struct AttnBf16Args {
-  CUtensorMap map_kv;      // 2-D {576, kv rows} bf16, box {64, 1}, 128B swizzle (gather4)
+  const __nv_bfloat16* kv; // latent KV rows [rows, 576] (contiguous, or pages of 64 rows)
+  int64_t ld_kv;           // elements between KV rows (a multiple of 8: 16-byte rows)
   const __nv_bfloat16* q;  // [n_q, 128, 576], 16-byte aligned rows
   int64_t ld_q;            // elements between query tokens
   const int32_t* idx;

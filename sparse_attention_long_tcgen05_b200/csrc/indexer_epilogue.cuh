@@ -13,9 +13,11 @@
 // with wq[j] = w[t,j] * sq[t] (the query's head weight times its FP8 scale) and
 // sk the key's FP8 scale. Multi-head ReLU gating as described in the
 // DeepSeek-V3.2-Exp report read-through (53ai.com), section "Innovative
-// architecture: core design of DSA". The four independent chains of eight
-// multiply-adds each hide the FMA latency with two epilogue warps per
-// scheduler; the packed form halves the multiply-add issue slots.
+// architecture: core design of DSA". Two independent chains per half of the
+// heads keep the multiply-add latency off the critical path; the packed form
+// halves the multiply-add issue slots. Each chain's operations and their order
+// are fixed by this definition, whether its inputs come from one TMEM load of
+// all 64 heads or two loads of 32.
 #pragma once
 
 #include <cstdint>
@@ -39,6 +41,44 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t w, uint64_t x, uint64_t acc) 
   return r;
 }
 
+// One step of a chain pair: (x, y) <- (w[0] * max(d0, 0) + x, w[1] * max(d1, 0) + y).
+__device__ __forceinline__ uint64_t chain_step(float w0, float w1, uint32_t d0, uint32_t d1,
+                                               uint64_t acc) {
+  return ffma2(pack_f32x2(w0, w1),
+               pack_f32x2(fmaxf(__uint_as_float(d0), 0.f), fmaxf(__uint_as_float(d1), 0.f)),
+               acc);
+}
+
+// Chains over 32 consecutive heads: x from dots[0..15] (weights wq[0..15]),
+// y from dots[16..31] (weights wq[16..31]), each in ascending head order.
+// Called with the dot products of heads 0..31 for chains A, B and of heads
+// 32..63 for chains C, D (raw TMEM words; wq 16-byte aligned shared memory).
+__device__ __forceinline__ void indexer_chains32(const uint32_t (&dots)[32],
+                                                 const float* __restrict__ wq, uint64_t& x,
+                                                 uint64_t& y) {
+  const float4* w4 = reinterpret_cast<const float4*>(wq);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 wa = w4[q];
+    const float4 wb = w4[4 + q];
+    x = chain_step(wa.x, wa.y, dots[4 * q + 0], dots[4 * q + 1], x);
+    y = chain_step(wb.x, wb.y, dots[16 + 4 * q + 0], dots[16 + 4 * q + 1], y);
+    x = chain_step(wa.z, wa.w, dots[4 * q + 2], dots[4 * q + 3], x);
+    y = chain_step(wb.z, wb.w, dots[16 + 4 * q + 2], dots[16 + 4 * q + 3], y);
+  }
+}
+
+// The score from the four finished chains and the key's scale.
+__device__ __forceinline__ float indexer_finish(uint64_t a, uint64_t b, uint64_t c, uint64_t d,
+                                                float sk) {
+  float ax, ay, bx, by, cx, cy, dx, dy;
+  unpack_f32x2(a, ax, ay);
+  unpack_f32x2(b, bx, by);
+  unpack_f32x2(c, cx, cy);
+  unpack_f32x2(d, dx, dy);
+  return (((ax + ay) + (bx + by)) + ((cx + cy) + (dx + dy))) * sk;
+}
+
 // lo: dot products of heads 0..31, hi: heads 32..63 (raw TMEM words);
 // wq: 64 head weights (16-byte aligned, shared memory).
 __device__ __forceinline__ float indexer_score_from_dots(const uint32_t (&lo)[32],
@@ -46,52 +86,9 @@ __device__ __forceinline__ float indexer_score_from_dots(const uint32_t (&lo)[32
                                                          const float* __restrict__ wq,
                                                          float sk) {
   uint64_t a = 0, b = 0, c = 0, d = 0;  // (+0.0f, +0.0f) pairs
-  const float4* w4 = reinterpret_cast<const float4*>(wq);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float4 wa = w4[q];
-    const float4 wb = w4[4 + q];
-    const float4 wc = w4[8 + q];
-    const float4 wd = w4[12 + q];
-    a = ffma2(pack_f32x2(wa.x, wa.y),
-              pack_f32x2(fmaxf(__uint_as_float(lo[4 * q + 0]), 0.f),
-                         fmaxf(__uint_as_float(lo[4 * q + 1]), 0.f)),
-              a);
-    b = ffma2(pack_f32x2(wb.x, wb.y),
-              pack_f32x2(fmaxf(__uint_as_float(lo[16 + 4 * q + 0]), 0.f),
-                         fmaxf(__uint_as_float(lo[16 + 4 * q + 1]), 0.f)),
-              b);
-    c = ffma2(pack_f32x2(wc.x, wc.y),
-              pack_f32x2(fmaxf(__uint_as_float(hi[4 * q + 0]), 0.f),
-                         fmaxf(__uint_as_float(hi[4 * q + 1]), 0.f)),
-              c);
-    d = ffma2(pack_f32x2(wd.x, wd.y),
-              pack_f32x2(fmaxf(__uint_as_float(hi[16 + 4 * q + 0]), 0.f),
-                         fmaxf(__uint_as_float(hi[16 + 4 * q + 1]), 0.f)),
-              d);
-    a = ffma2(pack_f32x2(wa.z, wa.w),
-              pack_f32x2(fmaxf(__uint_as_float(lo[4 * q + 2]), 0.f),
-                         fmaxf(__uint_as_float(lo[4 * q + 3]), 0.f)),
-              a);
-    b = ffma2(pack_f32x2(wb.z, wb.w),
-              pack_f32x2(fmaxf(__uint_as_float(lo[16 + 4 * q + 2]), 0.f),
-                         fmaxf(__uint_as_float(lo[16 + 4 * q + 3]), 0.f)),
-              b);
-    c = ffma2(pack_f32x2(wc.z, wc.w),
-              pack_f32x2(fmaxf(__uint_as_float(hi[4 * q + 2]), 0.f),
-                         fmaxf(__uint_as_float(hi[4 * q + 3]), 0.f)),
-              c);
-    d = ffma2(pack_f32x2(wd.z, wd.w),
-              pack_f32x2(fmaxf(__uint_as_float(hi[16 + 4 * q + 2]), 0.f),
-                         fmaxf(__uint_as_float(hi[16 + 4 * q + 3]), 0.f)),
-              d);
-  }
-  float ax, ay, bx, by, cx, cy, dx, dy;
-  unpack_f32x2(a, ax, ay);
-  unpack_f32x2(b, bx, by);
-  unpack_f32x2(c, cx, cy);
-  unpack_f32x2(d, dx, dy);
-  return (((ax + ay) + (bx + by)) + ((cx + cy) + (dx + dy))) * sk;
+  indexer_chains32(lo, wq, a, b);
+  indexer_chains32(hi, wq + 32, c, d);
+  return indexer_finish(a, b, c, d, sk);
 }
 
 }  // namespace dsa

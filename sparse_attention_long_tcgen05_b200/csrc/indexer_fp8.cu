@@ -153,13 +153,13 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
       mbar_init(&S.q_full[i], 1);
       mbar_init(&S.q_empty[i], 1);
       mbar_init(&S.acc_full[i], 1);
-      mbar_init(&S.acc_empty[i], kEpiThreads);
+      mbar_init(&S.acc_empty[i], kEpiWarps);
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&S.k_full[i], 1);
       // released by the MMAs' completion and by every epilogue thread that
       // reads the stage's key scales (half of them with one query per group)
-      mbar_init(&S.k_empty[i], 1 + (G == 1 ? kEpiThreads / 2 : kEpiThreads));
+      mbar_init(&S.k_empty[i], 1 + (G == 1 ? kEpiWarps / 2 : kEpiWarps));
     }
     mbar_init(&S.mma_drain, 1);
     fence_barrier_init();
@@ -353,7 +353,8 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
             const uint32_t kp = ks + half < kStages ? kph : kph ^ 1u;
             if (!mbar_wait_warp(&S.k_full[kss], kp, a.status, a.wait_ns)) { ok = false; break; }
             sk = S.sk[kss][sub * 32 + lane];
-            mbar_arrive(&S.k_empty[kss]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.k_empty[kss]);
           }
           if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status, a.wait_ns)) { ok = false; break; }
           tc_fence_after();
@@ -365,12 +366,14 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
             tmem_ld32(tbase + 32, r1);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&S.acc_empty[ab]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
             const float s0 = indexer_score_from_dots(r0, r1, &S.wq[0], sk);
             if (s < a.n_cols) srow[s] = s <= my_pos ? s0 : -INFINITY;
           } else {
             tc_fence_before();
-            mbar_arrive(&S.acc_empty[ab]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
           }
           for (int h = 0; h < nt; ++h)
             if (++ks == kStages) { ks = 0; kph ^= 1; }
@@ -397,7 +400,8 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
         // this tile's key scale (the stage also holds the key codes)
         if (!mbar_wait_warp(&S.k_full[ks], kph, a.status, a.wait_ns)) { ok = false; break; }
         const float sk = S.sk[ks][sub * 32 + lane];
-        mbar_arrive(&S.k_empty[ks]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.k_empty[ks]);
         if (++ks == kStages) { ks = 0; kph ^= 1; }
         if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status, a.wait_ns)) { ok = false; break; }
         tc_fence_after();
@@ -411,7 +415,8 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           tmem_ld32(tbase + 96, r3);
           tmem_wait_ld();
           tc_fence_before();
-          mbar_arrive(&S.acc_empty[ab]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
           const float s0 = indexer_score_from_dots(r0, r1, &S.wq[g0 * kHeads], sk);
           const float s1 = indexer_score_from_dots(r2, r3, &S.wq[(g0 + 1) * kHeads], sk);
           if (s < a.n_cols) {
@@ -424,12 +429,14 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           tmem_ld32(tbase + 32, r1);
           tmem_wait_ld();
           tc_fence_before();
-          mbar_arrive(&S.acc_empty[ab]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
           const float s0 = indexer_score_from_dots(r0, r1, &S.wq[g0 * kHeads], sk);
           if (s < a.n_cols) srow0[s] = s <= pos0 ? s0 : -INFINITY;
         } else {
           tc_fence_before();
-          mbar_arrive(&S.acc_empty[ab]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
         }
         if (++ab == 2) { ab = 0; aph ^= 1; }
       }

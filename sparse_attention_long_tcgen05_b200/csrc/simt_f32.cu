@@ -71,7 +71,8 @@ __device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) 
   return r;
 }
 
-// One CTA per (query, head).
+// One CTA per (query, head). Sparse: the query's k selected entries; dense
+// (idx null): entry j is key j for j <= pos, and k covers every key.
 __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnF32Args a) {
   extern __shared__ float sm[];
   float* qs = sm;                        // [d_qk]
@@ -84,10 +85,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnF32Arg
   const float* q = a.q + static_cast<int64_t>(qi) * a.ld_q + static_cast<int64_t>(h) * a.d_qk;
   for (int i = threadIdx.x; i < a.d_qk; i += blockDim.x) qs[i] = q[i];
   __syncthreads();
-  const int32_t* idx = a.idx + static_cast<int64_t>(qi) * a.ld_idx;
+  const int32_t* idx = a.idx ? a.idx + static_cast<int64_t>(qi) * a.ld_idx : nullptr;
   float mx = -INFINITY;
   for (int j = threadIdx.x; j < a.k; j += blockDim.x) {
-    const int e = idx[j];
+    const int e = idx ? idx[j] : (j <= pos ? j : -1);
     float z = -INFINITY;
     int row = -1;
     if (e > pos) {

@@ -215,6 +215,10 @@ __device__ __forceinline__ void stage_q_chunks(uint32_t taddr_q, const uint4* qr
   tmem_wait_st();
 }
 
+// kDense: dense causal attention (the baseline DSA replaces) -- query t attends
+// to every key 0..t, walked as consecutive 64-key blocks (rows computed, or one
+// 64-token page per block), masked past t in the last block; no index rows.
+template <bool kDense>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
   extern __shared__ uint8_t smem_raw[];
@@ -225,7 +229,9 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
   const uint32_t rank = cluster_ctarank();     // 0 or 1
   const uint32_t peer = rank ^ 1u;
   const int col0 = 256 * static_cast<int>(rank);
-  const int qi = blockIdx.x >> 1;
+  // dense: the longest queries (the latest positions) are launched first
+  const int qi = kDense ? a.keys.n_q - 1 - static_cast<int>(blockIdx.x >> 1)
+                        : static_cast<int>(blockIdx.x >> 1);
 
   int pos, seq = 0;
   bool q_ok = true;
@@ -239,7 +245,7 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
   // The planning warps issue their index-row loads first, so the loads
   // overlap the barrier set-up and the cluster sync below.
   int e_in[4] = {-1, -1, -1, -1};
-  if (warp < kPlanWarps) {
+  if (!kDense && warp < kPlanWarps) {
     const int32_t* irow = a.idx + static_cast<int64_t>(qi) * a.ld_idx;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -251,19 +257,19 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
 
   if (threadIdx.x == 0) {
     mbar_init(&S.plan_full, 1);
-    mbar_init(&S.q_full, 3 * 128);
+    mbar_init(&S.q_full, 12);          // softmax, send and receive warps (one arrival each)
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&S.kv_full[i], 1);   // the expect-tx arrival; gather4 bytes complete it
+      mbar_init(&S.kv_full[i], kGatherIssuers);   // one arrival per issuing warp
       mbar_init(&S.kv_empty[i], 1);
     }
     for (int i = 0; i < kRopeStages; ++i) {
-      mbar_init(&S.rope_full[i], 1);
+      mbar_init(&S.rope_full[i], kGatherIssuers);
       mbar_init(&S.rope_empty[i], 1);
     }
     mbar_init(&S.s_full, 1);
-    mbar_init(&S.s_empty, 2 * 128);   // softmax and send warps
+    mbar_init(&S.s_empty, 8);         // softmax and send warps (one arrival each)
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&S.p_full[b], 2 * 128);    // softmax and receive warps
+      mbar_init(&S.p_full[b], 8);          // softmax and receive warps (one arrival each)
       mbar_init(&S.p_empty[b], 2);         // this CTA's PV and the peer's PV are done
       mbar_init(&S.rxp_full[b], 1);
     }
@@ -274,7 +280,6 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
     fence_barrier_init();
     if (!q_ok) report(a.status, DSA_ERR_DEVICE_BOUNDS);
   }
-  if (threadIdx.x == 32) tma_prefetch_desc(&a.map_kv);
   if (warp == kMmaWarp) tmem_alloc(&S.tmem_base, kTmemCols);
   tc_fence_before();
   cluster_sync();  // barriers of both CTAs initialised before any remote arrive
@@ -283,7 +288,34 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
 
   if (warp < kSoftmaxWarp0) {
     regs_dec<kRegsSmall>();
-    if (warp < kPlanWarps) {
+    if (kDense && warp < kPlanWarps) {
+      // ---------------------------------------------------------- dense plan
+      // blocks 0 .. pos / 64; with paged keys every block's page id is checked
+      // first, and a query with a page id out of range is reported and left
+      // empty (zero output), since its keys cannot be read
+      int nblk = pos >= 0 ? (pos >> 6) + 1 : 0;
+      bool bad = false;
+      if (a.keys.paged) {
+        const int32_t* bt = a.keys.block_table + static_cast<int64_t>(seq) * a.keys.ld_block_table;
+        for (int b = warp * 32 + lane; b < nblk; b += kPlanWarps * 32) {
+          const int pg = __ldg(bt + b);
+          bad |= pg < 0 || pg >= a.keys.num_pages;
+        }
+      }
+      const bool wbad = __any_sync(0xffffffffu, bad);
+      if (lane == 0) S.bmask[warp][0] = wbad ? 1u : 0u;   // per-warp vote (unused when dense)
+      named_bar_sync(1, kPlanWarps * 32);
+      if (warp == 0) {
+        const bool any_bad =
+            __any_sync(0xffffffffu, lane < kPlanWarps && S.bmask[lane][0] != 0u);
+        if (lane == 0) {
+          if (any_bad && rank == 0) report(a.status, DSA_ERR_DEVICE_BOUNDS);
+          S.n_blocks = any_bad ? 0 : nblk;
+          mbar_arrive(&S.plan_full);
+        }
+      }
+    }
+    if (!kDense && warp < kPlanWarps) {
       // ---------------------------------------------------------- plan (warps 0-15)
       // warp w scans blocks 2w and 2w+1; e[2i + half] holds entry
       // (2w + i) * 64 + 32 half + lane
@@ -348,10 +380,15 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
     }
     if (warp != kMmaWarp) {
       // ---------------------------------------------------------- gather (19 issuing warps)
-      // Block j's 16 groups of 4 rows x 4 64-dim value chunks, plus the rope
-      // chunk of this CTA's 8 groups (keys 32 rank ..), are split over the
-      // issuers: issuer i requests pieces p = i, i + 19, ...; each lands as 4
-      // swizzled 128-byte rows.
+      // Block j's selected rows are copied with 16-byte cp.async straight into
+      // the 128-byte-swizzled K-major tiles the MMAs read: the CTA's 256 value
+      // columns of each of the 64 rows (one 512-byte row per warp instruction,
+      // lane l copying 16 bytes of 64-dim chunk l / 8) and the 64 rope columns
+      // of this CTA's 32 keys (four rows per instruction). The block's 72
+      // instructions go round-robin to the 19 issuing warps. A warp releases
+      // block j-1 to the MMA once its own copies of that block have landed (its
+      // cp.async groups), after a proxy fence that makes them visible to the
+      // tensor core; so each warp keeps two blocks of copies in flight.
       // Only issuer 0 waits on the ring's barriers; the other 18 warps sleep on
       // hardware named barrier 2 (taking no issue slots from the softmax warps)
       // and learn from a shared flag whether to go on, so all 19 always take
@@ -363,7 +400,23 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
       }
       named_bar_sync(2, kGatherIssuers * 32);
       const int n = S.gather_n;
-      const int n_req = (kBK / 4) * 4 + kBK / 8;
+      const int c_l = lane >> 3;            // 64-dim chunk (value) / row of four (rope)
+      const int i_l = lane & 7;             // 16-byte unit within the 128-byte row piece
+      const char* const kv_b = reinterpret_cast<const char*>(a.kv);
+      const int64_t ld_b = a.ld_kv * 2;
+      const int64_t val_off = static_cast<int64_t>(col0 + 64 * c_l + 8 * i_l) * 2;
+      const int64_t rope_off = static_cast<int64_t>(512 + 8 * i_l) * 2;
+      constexpr int n_items = kBK + kBK / 8;   // 64 value rows + 8 rope instructions
+      // copies of block jj have landed in this warp: release them to the MMA
+      auto release = [&](int jj) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&S.kv_full[jj % kStages]);
+          mbar_arrive(&S.rope_full[jj % kRopeStages]);
+        }
+      };
+      int issued = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
         const int rs = j % kRopeStages;
@@ -373,34 +426,49 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
           if (ok)
             ok = mbar_wait_warp(&S.rope_empty[rs],
                                 static_cast<uint32_t>((j / kRopeStages) & 1) ^ 1u, a.status);
-          if (lane == 0) {
-            if (ok) {
-              mbar_arrive_expect_tx(&S.kv_full[st], 4 * kChunkKV);
-              mbar_arrive_expect_tx(&S.rope_full[rs], kChunkKV / 2);
-            }
-            S.gather_go[j & 1] = ok ? 1 : 0;
-          }
+          if (lane == 0) S.gather_go[j & 1] = ok ? 1 : 0;
         }
         named_bar_sync(2, kGatherIssuers * 32);
         if (S.gather_go[j & 1] == 0) break;
-        if (lane == 0) {
-          const int* rb = S.rows + S.blk[j] * kBK;
-          for (int p = issuer; p < n_req; p += kGatherIssuers) {
-            if (p < (kBK / 4) * 4) {
-              const int g = p >> 2, c = p & 3;
-              const int4 r4 = *reinterpret_cast<const int4*>(rb + 4 * g);
-              tma_gather4(S.kv[st][c] + g * 512, &a.map_kv, col0 + 64 * c, r4.x, r4.y, r4.z,
-                          r4.w, &S.kv_full[st]);
-            } else {
-              const int gg = p - (kBK / 4) * 4;                  // 0..7
-              const int4 r4 = *reinterpret_cast<const int4*>(rb + 4 * (8 * rank + gg));
-              tma_gather4(S.rope[rs] + gg * 512, &a.map_kv, 512, r4.x, r4.y, r4.z, r4.w,
-                          &S.rope_full[rs]);
-            }
+        // KV row of row r of block j: the planned row (sparse); dense, the
+        // key j*64 + r (clamped to the query's last key; masked past it) or
+        // slot r of the block's 64-token page
+        const int* rb = kDense ? nullptr : S.rows + S.blk[j] * kBK;
+        int64_t dense_base = 0;
+        if (kDense)
+          dense_base = a.keys.paged
+                           ? static_cast<int64_t>(__ldg(a.keys.block_table +
+                                                        static_cast<int64_t>(seq) *
+                                                            a.keys.ld_block_table + j)) * kBK
+                           : static_cast<int64_t>(j) * kBK;
+        auto kv_row = [&](int r) -> int64_t {
+          if (!kDense) return rb[r];
+          if (a.keys.paged) return dense_base + r;
+          return min(dense_base + r, static_cast<int64_t>(pos));
+        };
+        const uint32_t kv_st = smem_u32(S.kv[st][c_l]);
+        const uint32_t rope_st = smem_u32(S.rope[rs]);
+        for (int p = issuer; p < n_items; p += kGatherIssuers) {
+          if (p < kBK) {
+            const int r = p;                                   // row of the block
+            const char* src = kv_b + kv_row(r) * ld_b + val_off;
+            cp_async16(kv_st + r * 128 + ((i_l ^ (r & 7)) << 4), src);
+          } else {
+            const int rr = 4 * (p - kBK) + c_l;                // row of this CTA's 32 keys
+            const char* src = kv_b + kv_row(32 * rank + rr) * ld_b + rope_off;
+            cp_async16(rope_st + rr * 128 + ((i_l ^ (rr & 7)) << 4), src);
           }
         }
-        __syncwarp();
+        cp_async_commit();
+        ++issued;
+        if (j > 0) {
+          cp_async_wait_group<1>();
+          release(j - 1);
+        }
       }
+      // the last block, and a drain after a give-up: every copy lands first
+      cp_async_wait_group<0>();
+      if (issued > 0) release(issued - 1);
     } else {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc_qk = make_idesc(kBK, 1, 1, 0, 0);   // bf16, A (TMEM) and B K-major
@@ -491,7 +559,8 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
       const int cs[3] = {0, 3, 4};   // the send and receive warps stage 1 and 2
       stage_q_chunks(tmem_base + lane_q + kColQ, qrow, col0, cs);
       tc_fence_before();
-      mbar_arrive(&S.q_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.q_full);
     }
     bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
     const int n = ok ? S.n_blocks : 0;
@@ -512,7 +581,13 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n && ok; ++j) {
         const int b = j & 1;                       // P tile of this block
-        const uint32_t mk = S.mask[j][hh];         // valid keys among this thread's 32
+        uint32_t mk;                               // valid keys among this thread's 32
+        if (kDense) {
+          const int nv = pos - (j * kBK + 32 * hh) + 1;
+          mk = nv >= 32 ? 0xffffffffu : (nv <= 0 ? 0u : (1u << nv) - 1u);
+        } else {
+          mk = S.mask[j][hh];
+        }
         // own partial S of the block
         if (!mbar_wait_warp(&S.s_full, static_cast<uint32_t>(j & 1), a.status)) {
           ok = false;
@@ -523,7 +598,8 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
         tmem_ld16x2_32(t_lane + kColS, v);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&S.s_empty);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.s_empty);
         // the peer's partial for our heads
         if (warp == kSoftmaxWarp0 && lane == 0) mbar_arrive_expect_tx(&S.rxs_full, kRxSBytes);
         if (!mbar_wait_cluster_warp(&S.rxs_full, static_cast<uint32_t>(j & 1), a.status)) {
@@ -595,8 +671,10 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
           *reinterpret_cast<uint4*>(prow + cc) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
         l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-        // P rows and factors visible to the async proxy (our MMA, the copy to the peer)
+        // P rows and factors visible to the async proxy (our MMA, the copy to
+        // the peer); any O rescale of this thread ordered before the release
         fence_proxy_async_smem();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) {
           const uint32_t bb = static_cast<uint32_t>(b);
@@ -605,9 +683,8 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
                                rxp_full_peer);
           bulk_copy_to_cluster(alpha_peer0 + 256u * bb, smem_u32(&S.tx_alpha[b][16 * s]), 64,
                                rxp_full_peer);
+          mbar_arrive(&S.p_full[b]);
         }
-        tc_fence_before();
-        mbar_arrive(&S.p_full[b]);
       }
       // epilogue: O / l -> bf16 for own heads, lse; the peer gets l for its rows
       const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
@@ -642,7 +719,8 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
       const int cs[1] = {warp < kRecvWarp0 ? 1 : 2};
       stage_q_chunks(tmem_base + lane_q + kColQ, qrow, col0, cs);
       tc_fence_before();
-      mbar_arrive(&S.q_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.q_full);
     }
     bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
     const int n = ok ? S.n_blocks : 0;
@@ -665,7 +743,8 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
         tmem_ld16x2_32(t_lane + kColS, v);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&S.s_empty);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.s_empty);
         // the peer has read block j-1 out of its rx_s (so our copy out of tx_s is done)
         if (!mbar_wait_cluster_warp(&S.rxs_free, static_cast<uint32_t>((j & 1) ^ 1),
                                     a.status)) {
@@ -708,7 +787,8 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
         }
         fence_proxy_async_smem();   // the peer's rows, seen here, before the MMA reads them
         tc_fence_before();
-        mbar_arrive(&S.p_full[b]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.p_full[b]);
       }
       if (warp == kRecvWarp0 && lane == 0) mbar_arrive_expect_tx(&S.l_full, 64 * 4);
       const bool l_ok = mbar_wait_cluster_warp(&S.l_full, 0, a.status);
@@ -737,11 +817,19 @@ cudaError_t launch_attn_bf16(const AttnBf16Args& a, cudaStream_t stream) {
   if (a.keys.n_q <= 0) return cudaSuccess;
   if (a.k > kMaxK) return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(sparse_mqa_bf16_kernel,
+  if (a.idx == nullptr) {   // dense causal attention
+    cudaError_t e = cudaFuncSetAttribute(sparse_mqa_bf16_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    sparse_mqa_bf16_kernel<true><<<2 * a.keys.n_q, kThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+  }
+  cudaError_t e = cudaFuncSetAttribute(sparse_mqa_bf16_kernel<false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  sparse_mqa_bf16_kernel<<<2 * a.keys.n_q, kThreads, smem, stream>>>(a);
+  sparse_mqa_bf16_kernel<false><<<2 * a.keys.n_q, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -34,7 +34,7 @@ DSA_OP_SELECT = 4
 EXPORTED = ["dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_fwd", "dsa_select", "dsa_forward",
             "dsa_workspace_size", "dsa_check_status", "dsa_status_string",
             "dsa_last_cuda_error", "dsa_launch_counter", "dsa_version", "dsa_select_noalloc",
-            "dsa_set_wait_limit_ns"]
+            "dsa_set_wait_limit_ns", "dsa_dense_mqa_fwd"]
 
 
 class DsaError(RuntimeError):
@@ -80,6 +80,7 @@ def _load():
         "dsa_topk": [P, I64, P, I32, I32, P, I64, P],
         "dsa_sparse_mqa_fwd": [ctypes.POINTER(AttnIn), P, I64, I32, P, P, P, SZ, P],
         "dsa_select": [ctypes.POINTER(IndexerIn), I32, P, I64, P, SZ, P],
+        "dsa_dense_mqa_fwd": [ctypes.POINTER(AttnIn), P, P, P],
         "dsa_forward": [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), I32, P, P, P, P, SZ, P],
         "dsa_launch_counter": [],
         "dsa_set_wait_limit_ns": [I64],
@@ -210,6 +211,12 @@ def dsa_sparse_mqa_fwd(attn: _Keep, idx: torch.Tensor, k: int, out: torch.Tensor
                                   _ptr(out), _ptr(lse), _ptr(ws),
                                   0 if ws is None else ws.numel() * ws.element_size(),
                                   _stream(stream)), "dsa_sparse_mqa_fwd")
+
+
+def dsa_dense_mqa_fwd(attn: _Keep, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                      stream=None):
+    _check(LIB.dsa_dense_mqa_fwd(ctypes.byref(attn.struct), _ptr(out), _ptr(lse),
+                                 _stream(stream)), "dsa_dense_mqa_fwd")
 
 
 def dsa_select(ind: _Keep, k: int, idx: torch.Tensor, ws: torch.Tensor, stream=None):
