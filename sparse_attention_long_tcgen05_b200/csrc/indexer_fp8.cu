@@ -134,9 +134,14 @@ __device__ __forceinline__ int page_of(const IndexerFp8Args& a, int seq, int p,
   return page;
 }
 
+// kLimitArg: the pipeline waits take their bound from a.wait_ns (a launch after
+// the caller changed the bound); otherwise the default bound is a compile-time
+// constant and each wait's suspend hint an immediate.
+template <bool kLimitArg>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks, int n_tiles,
                    int tpu, int n_units) {
+  const uint64_t wait_ns = kLimitArg ? a.wait_ns : kWaitLimitNs;
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                      ~uintptr_t(1023));
@@ -153,13 +158,13 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
       mbar_init(&S.q_full[i], 1);
       mbar_init(&S.q_empty[i], 1);
       mbar_init(&S.acc_full[i], 1);
-      mbar_init(&S.acc_empty[i], kEpiWarps);
+      mbar_init(&S.acc_empty[i], kEpiThreads);
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&S.k_full[i], 1);
       // released by the MMAs' completion and by every epilogue thread that
       // reads the stage's key scales (half of them with one query per group)
-      mbar_init(&S.k_empty[i], 1 + (G == 1 ? kEpiWarps / 2 : kEpiWarps));
+      mbar_init(&S.k_empty[i], 1 + (G == 1 ? kEpiThreads / 2 : kEpiThreads));
     }
     mbar_init(&S.mma_drain, 1);
     fence_barrier_init();
@@ -197,11 +202,13 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
       const int qb = it & 1;
       const uint32_t qph = (it >> 1) & 1;
       if (first) {
-        if (!mbar_wait_warp(&S.q_empty[qb], qph ^ 1, a.status, a.wait_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&S.q_empty[qb], qph ^ 1, a.status, wait_ns)) { ok = false; break; }
         if (lane == 0) {
           mbar_arrive_expect_tx(&S.q_full[qb], U.ng * kQBytes);
-          for (int i = 0; i < U.ng; ++i)
-            tma_load_3d(S.q[qb] + i * kQBytes, &a.map_q, 0, 0, U.qi[i], &S.q_full[qb]);
+#pragma unroll
+          for (int i = 0; i < kMaxG; ++i)   // constant indices keep U in registers
+            if (i < U.ng)
+              tma_load_3d(S.q[qb] + i * kQBytes, &a.map_q, 0, 0, U.qi[i], &S.q_full[qb]);
         }
         ++q_fills[qb];
       }
@@ -212,7 +219,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           pg = page_of(a, U.seq0, p, first);
       }
       for (int t = U.t0; t < U.t_end; ++t) {
-        if (!mbar_wait_warp(&S.k_empty[ks], kph ^ 1, a.status, a.wait_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&S.k_empty[ks], kph ^ 1, a.status, wait_ns)) { ok = false; break; }
         const int i0 = 2 * (t - U.t0);
         const int pg0 = __shfl_sync(0xffffffffu, pg, i0 & 31);
         const int pg1 = __shfl_sync(0xffffffffu, pg, (i0 + 1) & 31);
@@ -259,7 +266,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
         const Unit U = get_unit(a, G, n_chunks, n_tiles, tpu, u, false);
         const int qb = it & 1;
         const uint32_t qph = (it >> 1) & 1;
-        if (!mbar_wait(&S.q_full[qb], qph, a.status, a.wait_ns)) break;
+        if (!mbar_wait(&S.q_full[qb], qph, a.status, wait_ns)) break;
         tc_fence_after();
         const uint64_t bdesc = sw128_desc(smem_u32(S.q[qb]), 16, 1024);
         if (G == 1) {
@@ -267,11 +274,11 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           // 128-column accumulator
           for (int t = U.t0; t < U.t_end && ok; t += 2) {
             const int nt = min(2, U.t_end - t);
-            if (!mbar_wait(&S.acc_empty[ab], aph ^ 1, a.status, a.wait_ns)) { ok = false; break; }
+            if (!mbar_wait(&S.acc_empty[ab], aph ^ 1, a.status, wait_ns)) { ok = false; break; }
             for (int h = 0; h < nt && ok; ++h) {
               const int kss = ks + h < kStages ? ks + h : ks + h - kStages;
               const uint32_t kp = ks + h < kStages ? kph : kph ^ 1u;
-              if (!mbar_wait(&S.k_full[kss], kp, a.status, a.wait_ns)) ok = false;
+              if (!mbar_wait(&S.k_full[kss], kp, a.status, wait_ns)) ok = false;
             }
             if (!ok) break;
             tc_fence_after();
@@ -294,7 +301,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
         }
         for (int t = U.t0; t < U.t_end; ++t) {
           if (!mbar_wait(&S.k_full[ks], kph, a.status) ||
-              !mbar_wait(&S.acc_empty[ab], aph ^ 1, a.status, a.wait_ns)) { ok = false; break; }
+              !mbar_wait(&S.acc_empty[ab], aph ^ 1, a.status, wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = sw128_desc(smem_u32(S.k[ks]), 16, 1024);
           const uint32_t d = tmem_base + static_cast<uint32_t>(ab * N);
@@ -330,7 +337,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
       named_bar_sync(1, kEpiThreads);
       for (int i = et; i < U.ng * kHeads; i += kEpiThreads) {
         const int g = i / kHeads;
-        const int qi = U.qi[g];
+        const int qi = g == 0 ? U.qi[0] : g == 1 ? U.qi[1] : g == 2 ? U.qi[2] : U.qi[3];
         S.wq[i] = a.w[static_cast<int64_t>(qi) * a.ld_w + (i % kHeads)] * a.q_scale[qi];
       }
       named_bar_sync(1, kEpiThreads);
@@ -351,12 +358,11 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           if (mine) {
             const int kss = ks + half < kStages ? ks + half : ks + half - kStages;
             const uint32_t kp = ks + half < kStages ? kph : kph ^ 1u;
-            if (!mbar_wait_warp(&S.k_full[kss], kp, a.status, a.wait_ns)) { ok = false; break; }
+            if (!mbar_wait_warp(&S.k_full[kss], kp, a.status, wait_ns)) { ok = false; break; }
             sk = S.sk[kss][sub * 32 + lane];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.k_empty[kss]);
+            mbar_arrive(&S.k_empty[kss]);
           }
-          if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status, a.wait_ns)) { ok = false; break; }
+          if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status, wait_ns)) { ok = false; break; }
           tc_fence_after();
           if (mine) {
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) +
@@ -366,14 +372,12 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
             tmem_ld32(tbase + 32, r1);
             tmem_wait_ld();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
+            mbar_arrive(&S.acc_empty[ab]);
             const float s0 = indexer_score_from_dots(r0, r1, &S.wq[0], sk);
             if (s < a.n_cols) srow[s] = s <= my_pos ? s0 : -INFINITY;
           } else {
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
+            mbar_arrive(&S.acc_empty[ab]);
           }
           for (int h = 0; h < nt; ++h)
             if (++ks == kStages) { ks = 0; kph ^= 1; }
@@ -398,12 +402,11 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           continue;
         }
         // this tile's key scale (the stage also holds the key codes)
-        if (!mbar_wait_warp(&S.k_full[ks], kph, a.status, a.wait_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&S.k_full[ks], kph, a.status, wait_ns)) { ok = false; break; }
         const float sk = S.sk[ks][sub * 32 + lane];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.k_empty[ks]);
+        mbar_arrive(&S.k_empty[ks]);
         if (++ks == kStages) { ks = 0; kph ^= 1; }
-        if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status, a.wait_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&S.acc_full[ab], aph, a.status, wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) +
                                static_cast<uint32_t>(ab * N + g0 * kHeads);
@@ -415,8 +418,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           tmem_ld32(tbase + 96, r3);
           tmem_wait_ld();
           tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
+          mbar_arrive(&S.acc_empty[ab]);
           const float s0 = indexer_score_from_dots(r0, r1, &S.wq[g0 * kHeads], sk);
           const float s1 = indexer_score_from_dots(r2, r3, &S.wq[(g0 + 1) * kHeads], sk);
           if (s < a.n_cols) {
@@ -429,14 +431,12 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
           tmem_ld32(tbase + 32, r1);
           tmem_wait_ld();
           tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
+          mbar_arrive(&S.acc_empty[ab]);
           const float s0 = indexer_score_from_dots(r0, r1, &S.wq[g0 * kHeads], sk);
           if (s < a.n_cols) srow0[s] = s <= pos0 ? s0 : -INFINITY;
         } else {
           tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
+          mbar_arrive(&S.acc_empty[ab]);
         }
         if (++ab == 2) { ab = 0; aph ^= 1; }
       }
@@ -484,8 +484,9 @@ cudaError_t launch_indexer_fp8(const IndexerFp8Args& a, int num_sms, bool pdl,
   if (n_units_ll > 0x7fffffffLL) return cudaErrorInvalidValue;
   const int n_units = static_cast<int>(n_units_ll);
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(indexer_fp8_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const bool limit_arg = a.wait_ns != kWaitLimitNs;
+  auto kernel = limit_arg ? indexer_fp8_kernel<true> : indexer_fp8_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -498,7 +499,7 @@ cudaError_t launch_indexer_fp8(const IndexerFp8Args& a, int num_sms, bool pdl,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, indexer_fp8_kernel, a, G, n_chunks, n_tiles, tpu, n_units);
+  return cudaLaunchKernelEx(&cfg, kernel, a, G, n_chunks, n_tiles, tpu, n_units);
 }
 
 }  // namespace dsa
