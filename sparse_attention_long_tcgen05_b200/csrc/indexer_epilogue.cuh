@@ -10,7 +10,8 @@
 //   j with a packed fused multiply-add:  (x, y) <- (wq[j] * max(d_j, 0) + x,
 //                                                  wq[j+1] * max(d_j+1, 0) + y)
 //
-// with wq[j] = w[t,j] * sq[t] (the query's head weight times its FP8 scale) and
+// with wq[j] = w[t,j] * sq[t] (the query's head weight times its FP8 scale;
+// staged halved for odd j, see chain_step) and
 // sk the key's FP8 scale. Multi-head ReLU gating as described in the
 // DeepSeek-V3.2-Exp report read-through (53ai.com), section "Innovative
 // architecture: core design of DSA". Two independent chains per half of the
@@ -42,11 +43,15 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t w, uint64_t x, uint64_t acc) 
 }
 
 // One step of a chain pair: (x, y) <- (w[0] * max(d0, 0) + x, w[1] * max(d1, 0) + y).
+// The odd head's ReLU is evaluated as d + |d| = 2 max(d, 0) with its weight
+// staged at half (wq[j] = w[t,j] sq[t] / 2 for odd j): both factors are exact
+// (scaling by a power of two), so the product and the fused multiply-add round
+// exactly as w * max(d, 0) would, while the add runs on the FMA pipe and the
+// max of the even head on the ALU pipe, which takes a max at half rate.
 __device__ __forceinline__ uint64_t chain_step(float w0, float w1, uint32_t d0, uint32_t d1,
                                                uint64_t acc) {
-  return ffma2(pack_f32x2(w0, w1),
-               pack_f32x2(fmaxf(__uint_as_float(d0), 0.f), fmaxf(__uint_as_float(d1), 0.f)),
-               acc);
+  const float x0 = __uint_as_float(d0), x1 = __uint_as_float(d1);
+  return ffma2(pack_f32x2(w0, w1), pack_f32x2(fmaxf(x0, 0.f), x1 + fabsf(x1)), acc);
 }
 
 // Chains over 32 consecutive heads: x from dots[0..15] (weights wq[0..15]),

@@ -338,7 +338,9 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
       for (int i = et; i < U.ng * kHeads; i += kEpiThreads) {
         const int g = i / kHeads;
         const int qi = g == 0 ? U.qi[0] : g == 1 ? U.qi[1] : g == 2 ? U.qi[2] : U.qi[3];
-        S.wq[i] = a.w[static_cast<int64_t>(qi) * a.ld_w + (i % kHeads)] * a.q_scale[qi];
+        // odd heads staged at half weight: their ReLU is taken as d + |d| (chain_step)
+        S.wq[i] = a.w[static_cast<int64_t>(qi) * a.ld_w + (i % kHeads)] * a.q_scale[qi] *
+                  ((i & 1) ? 0.5f : 1.f);
       }
       named_bar_sync(1, kEpiThreads);
       if (G == 1) {

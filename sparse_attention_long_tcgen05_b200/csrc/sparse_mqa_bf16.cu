@@ -14,15 +14,21 @@
 // the 576 key dimensions: CTA0 owns dims [0,256), CTA1 [256,512), and the 64 rope
 // dims are split by key (see below). Each CTA
 //   - keeps its slice of Q in TMEM (the MMA's A operand read from tensor
-//     memory) and gathers only its column range of the selected rows with TMA
-//     tile::gather4 (four 128-byte row pieces per request, 128B-swizzled on
-//     arrival, no multicast), so the pair reads each selected row once;
+//     memory) and gathers only its column range of the selected rows with
+//     per-thread 16-byte cp.async copies written straight into the
+//     128-byte-swizzled tiles the MMAs read, so the pair reads each selected
+//     row once (TMA tile::gather4 requests, one per four 128-byte row pieces,
+//     were slower: their issue rate, ~35 cycles per request, set the pace);
 //   - computes a partial S_r = Q[:, dims_r] K[:, dims_r]^T for all 128 heads
 //     (M=128, N=64 keys) into TMEM;
 //   - owns the softmax of 64 of the heads. TMEM lane 32s+i (i < 16) of SM
 //     sub-partition s holds one of its own heads, lane 32s+16+i one of the
 //     peer's; Q rows are staged in that order, so S, P and O rows follow it.
-//     The CTA sends the peer the 16 KB partial S of the peer's heads, adds
+//     The CTA sends the peer the 8 KB partial S of the peer's heads (fp16: the
+//     partials of a 288-dim dot product of bf16 rows stay far inside fp16's
+//     range, and its 11-bit rounding lies well below the bf16 rounding P gets
+//     right after; halving these bytes cut the 128K attention from 146 to
+//     138 ms on B200), adds
 //     the peer's partial for its own heads, runs the online softmax and
 //     writes the bf16 P rows of its heads into its own P tile, from where
 //     they are copied into the peer's (8 KB), together with the per-head
@@ -33,7 +39,7 @@
 //   - accumulates its half of the value columns, O[:, 256r : 256r+256] += P V_r
 //     for all 128 heads, where V_r lies inside its own gathered columns.
 // Measured on B200, cluster shared-memory traffic runs at ~20 B/cycle per SM
-// and direction, so the exchange is kept to the 24 KB per 64-key block that
+// and direction, so the exchange is kept to the 16 KB per 64-key block that
 // the split requires, and QK^T of block j+1 is issued as soon as S_j has been
 // read, so that the partial S of block j+1 travels while block j's softmax runs.
 // The softmax keeps a stale running max and rescales O in TMEM only when the
@@ -44,17 +50,20 @@
 // Roles per CTA (1024 threads, 8 warps per SM sub-partition):
 //   warps 0-15   plan (each scans two 64-entry blocks of the query's index row:
 //                physical rows, valid masks);
-//   warps 0-15, 17-19  issue the gather requests (lane 0 of each);
+//   warps 0-15, 17-19  copy the selected rows (all lanes, cp.async);
 //   warp 16      owns TMEM and issues the MMAs;
 //   warps 20-23  softmax of the CTA's own heads (TMEM lanes 32s .. 32s+15);
-//   warps 24-27  send the peer's partial S (lanes 32s+16 .. 32s+31);
+//   warps 24-27  send the peer's partial S (lanes 32s+16 .. 32s+31), as fp16;
 //   warps 28-31  take in the peer's P rows and rescale factors, rescale the
 //                peer's O rows here, and write those rows at the end.
 // The 64 rope dims are needed only by QK^T. Each CTA gathers them for its own
 // 32 keys of a block (CTA r: keys 32r .. 32r+31) into a ring of their own,
 // released as soon as QK^T has read it, and adds their term to those 32
-// columns of its partial S; with 4 value chunks plus half a rope chunk each,
-// the pair issues 72 gather requests per CTA and block.
+// columns of its partial S; with 64 value-row pieces of 512 bytes plus 8
+// instructions of four 128-byte rope pieces, each CTA issues 72 warp-wide copy
+// instructions per block.
+#include <cuda_fp16.h>
+
 #include "dsa_common.cuh"
 #include "dsa_kernels.h"
 
@@ -69,12 +78,11 @@ constexpr int kChunkKV = kBK * 128;  // one 64-dim chunk of a key block: 64 rows
 constexpr int kMaxK = 2048;
 constexpr int kMaxBlocks = kMaxK / kBK;
 static_assert(kMaxBlocks <= 32, "one lane of a warp per key block in the plan's compaction");
-// Warp roles. One TMA tile::gather4 request moves four 128-byte row pieces
-// and keeps its issuing warp busy ~90 cycles; measured on B200, the gather
-// rate grows with the number of issuing warps (not lanes), so 19 warps issue.
+// Warp roles. 19 warps copy the selected rows (a block's 72 row-piece
+// instructions round-robin over them).
 constexpr int kPlanWarps = 16;       // warps 0-15 scan the index row (two blocks each)
 constexpr int kMmaWarp = 16;
-constexpr int kGatherIssuers = 19;   // warps 0-15 and 17-19 issue gather4 requests
+constexpr int kGatherIssuers = 19;   // warps 0-15 and 17-19 copy the selected rows
 constexpr int kSoftmaxWarp0 = 20;    // 20..23
 constexpr int kSendWarp0 = 24;       // 24..27
 constexpr int kRecvWarp0 = 28;       // 28..31
@@ -91,15 +99,15 @@ constexpr uint32_t kColO = 0;
 constexpr uint32_t kColS = 256;
 constexpr uint32_t kColQ = 320;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr uint32_t kRxSBytes = 64 * kBK * 4;        // the peer's partial S of our 64 heads
+constexpr uint32_t kRxSBytes = 64 * kBK * 2;        // the peer's partial S of our 64 heads (fp16)
 constexpr uint32_t kRxPBytes = 64 * 128 + 64 * 4;   // the peer's 64 P rows + rescale factors
 
 struct __align__(1024) Smem {
   uint8_t kv[kStages][4][kChunkKV];           // 128 KB value-chunk ring
   uint8_t rope[kRopeStages][kChunkKV / 2];    // 8 KB: rope dims of this CTA's 32 keys
   uint8_t p[2][kH * 128];                     // 2 x 16 KB: P [128 rows x 64 keys] bf16
-  float rx_s[64 * kBK];                       // 16 KB: the peer's partial S of our heads
-  float tx_s[64 * kBK];                       // 16 KB: our partial S of the peer's heads
+  uint32_t rx_s[64 * kBK / 2];                // 8 KB: the peer's partial S of our heads (fp16 pairs)
+  uint32_t tx_s[64 * kBK / 2];                // 8 KB: our partial S of the peer's heads (fp16 pairs)
   int32_t rows[kMaxK];                        // KV row of every index entry (0 if invalid)
   uint32_t bmask[kMaxBlocks][2];              // valid entries of block b
   uint32_t mask[kMaxBlocks][2];               // valid entries of the j-th non-empty block
@@ -607,14 +615,17 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
           break;
         }
         float x[32];
-        const float4* rp = reinterpret_cast<const float4*>(S.rx_s + o * kBK);
+        const uint4* rp = reinterpret_cast<const uint4*>(S.rx_s + o * (kBK / 2));
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float4 pv = rp[(8 * hh + c) ^ static_cast<int>(sw)];
-          x[4 * c + 0] = __uint_as_float(v[4 * c + 0]) + pv.x;
-          x[4 * c + 1] = __uint_as_float(v[4 * c + 1]) + pv.y;
-          x[4 * c + 2] = __uint_as_float(v[4 * c + 2]) + pv.z;
-          x[4 * c + 3] = __uint_as_float(v[4 * c + 3]) + pv.w;
+        for (int c = 0; c < 4; ++c) {
+          const uint4 pv = rp[(4 * hh + c) ^ static_cast<int>(sw)];
+          const uint32_t w4[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[i]));
+            x[8 * c + 2 * i] = __uint_as_float(v[8 * c + 2 * i]) + f.x;
+            x[8 * c + 2 * i + 1] = __uint_as_float(v[8 * c + 2 * i + 1]) + f.y;
+          }
         }
         // block row max over both key halves (threads t and t ^ 16 share a head)
         if (mk != 0xffffffffu) {
@@ -728,10 +739,10 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
       // ---------------------------------------------------------- send the peer's partial S
       // thread t: the peer's head o in TMEM lane 32s + 16 + (t & 15), keys 32 hh .. +31
       const uint32_t t_lane = tmem_base + lane_q + (16u << 16);
-      uint8_t* tx_row = reinterpret_cast<uint8_t*>(S.tx_s + o * kBK);
+      uint8_t* tx_row = reinterpret_cast<uint8_t*>(S.tx_s + o * (kBK / 2));
       // this warp's rows 16s .. 16s+15 of tx_s go to the same rows of the peer's rx_s
-      const uint32_t tx_warp = smem_u32(S.tx_s + 16 * s * kBK);
-      const uint32_t rxs_peer_warp = mapa_shared(smem_u32(S.rx_s + 16 * s * kBK), peer);
+      const uint32_t tx_warp = smem_u32(S.tx_s + 16 * s * (kBK / 2));
+      const uint32_t rxs_peer_warp = mapa_shared(smem_u32(S.rx_s + 16 * s * (kBK / 2)), peer);
       const uint32_t rxs_full_peer = mapa_shared(smem_u32(&S.rxs_full), peer);
       for (int j = 0; j < n && ok; ++j) {
         if (!mbar_wait_warp(&S.s_full, static_cast<uint32_t>(j & 1), a.status)) {
@@ -751,15 +762,21 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
           ok = false;
           break;
         }
+        uint32_t hv[16];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t cc = (static_cast<uint32_t>(8 * hh + c) ^ sw) << 4;
-          *reinterpret_cast<uint4*>(tx_row + cc) = make_uint4(v[4 * c], v[4 * c + 1],
-                                                              v[4 * c + 2], v[4 * c + 3]);
+        for (int i = 0; i < 16; ++i) {
+          const __half2 h = __floats2half2_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          hv[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t cc = (static_cast<uint32_t>(4 * hh + c) ^ sw) << 4;
+          *reinterpret_cast<uint4*>(tx_row + cc) = make_uint4(hv[4 * c], hv[4 * c + 1],
+                                                              hv[4 * c + 2], hv[4 * c + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) bulk_copy_to_cluster(rxs_peer_warp, tx_warp, 16 * kBK * 4, rxs_full_peer);
+        if (lane == 0) bulk_copy_to_cluster(rxs_peer_warp, tx_warp, 16 * kBK * 2, rxs_full_peer);
       }
     } else {
       // ---------------------------------------------------------- the peer's P rows
