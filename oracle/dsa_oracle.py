@@ -16,7 +16,8 @@ Every step is the plain definition, in float64, with numpy library primitives
   4. MQA-mode attention of all query heads over the selected shared latent KV
      rows (V = the first d_v columns of the KV row), with the exact softmax and
      its log-sum-exp;
-  5. dense causal attention, used only to pin step 4.
+  5. dense causal attention, used to pin step 4 and as the dense baseline;
+  6. the indexer's KL training signal over a key set.
 
 Sources (web pages on DeepSeek-V3.2 / V3.2-Exp):
   [53ai]  "DeepSeek-V3.2-Exp 技术报告解读" (53ai.com), section
@@ -26,6 +27,8 @@ Sources (web pages on DeepSeek-V3.2 / V3.2-Exp):
           and "第二步：Fine-grained Token Selection".
   [pb]    paperbridge.wiki summary of arXiv 2512.02556, sections
           "密集注意力" (dense attention) and "DeepSeek Sparse Attention".
+  [amaranth] engineering report on wiki-for-amaranth, section "DeepSeek
+          Sparse Attention (DSA)" (indexer trained by a KL loss; stages A, B).
   [ocp]   OCP 8-bit floating point specification, E4M3 format (the pages only
           say "FP8"; the e4m3 variant and per-token scales are the workload's).
 
@@ -160,6 +163,53 @@ def dense_causal_attention(q, k, v, scale):
     for t in range(L):
         out[t], lse[t], _ = attend(q[t], k[: t + 1], v[: t + 1], scale)
     return out, lse
+
+
+# ------------------------------------------- indexer KL training signal
+
+def indexer_kl_row(q_t, keys, scale, scores):
+    """Training signal of the lightning indexer for one query token over a key
+    set (the selected keys in sparse training; every preceding key in the dense
+    warm-up). [amaranth] section "DeepSeek Sparse Attention (DSA)" and [juhe]
+    "阶段一：Dense Warm-up" / "阶段二：Sparse Training": the indexer learns to
+    match the main attention's distribution through a KL-divergence loss;
+    [53ai] "持续预训练：逐步优化稀疏机制" (continued pre-training): in sparse
+    training the KL term is kept with only the top-k keys selected.
+
+    The main attention distribution is every head's softmax over the keys,
+    averaged over the heads (so it sums to 1); the indexer's is the softmax of
+    its scores over the same keys. Returns (p, r, kl, grad): p the target, r
+    the indexer distribution, kl = KL(p || r) = sum_i p_i (log p_i - log r_i),
+    and grad = d kl / d scores = r - p (p taken as fixed).
+    q_t [H, d_qk], keys [n, d_qk], scores [n]."""
+    q_t = np.asarray(q_t, dtype=np.float64)
+    keys = np.asarray(keys, dtype=np.float64)
+    _, _, probs = attend(q_t, keys, keys[:, :1], scale)     # [H, n] per-head softmax
+    p = probs.mean(axis=0)
+    s = np.asarray(scores, dtype=np.float64)
+    e = np.exp(s - s.max())
+    r = e / e.sum()
+    pos = p > 0
+    kl = float(np.sum(p[pos] * (np.log(p[pos]) - np.log(r[pos]))))
+    return p, r, kl, r - p
+
+
+def indexer_kl_rows(q, kv, idx, rows, scale, sel_scores):
+    """indexer_kl_row for each query row in ``rows`` over its selection
+    idx[r] (entries < 0 skipped) with the indexer scores of those entries,
+    sel_scores[r] (same positions as idx[r]). Returns (p, kl, grad) with p and
+    grad laid out like idx (0 at skipped entries)."""
+    idx = np.asarray(idx)
+    p_out = np.zeros(idx.shape)
+    g_out = np.zeros(idx.shape)
+    kl = np.zeros(len(rows))
+    for r, row in enumerate(rows):
+        m = idx[r] >= 0
+        keys = np.asarray(kv)[idx[r][m]]
+        p, _, kl[r], g = indexer_kl_row(q[row], keys, scale, np.asarray(sel_scores)[r][m])
+        p_out[r, m] = p
+        g_out[r, m] = g
+    return p_out, kl, g_out
 
 
 # ------------------------------------------------------------- paged caches

@@ -254,6 +254,86 @@ def check_attention_properties(attend, sparse_mqa_row):
     assert np.allclose(la, lb, rtol=1e-12, atol=1e-12)
 
 
+def _kl_case(seed=0, H=3, n=7, d=5):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((H, d)), rng.standard_normal((n, d)), 0.7,
+            rng.standard_normal(n) * 2.0)
+
+
+def check_kl_gradient_finite_differences(kl_row):
+    """d kl / d scores from central differences of the loss itself."""
+    q, keys, scale, sc = _kl_case(1)
+    _, _, _, g = kl_row(q, keys, scale, sc)
+    eps = 1e-6
+    fd = np.zeros_like(sc)
+    for i in range(sc.size):
+        e = np.zeros_like(sc)
+        e[i] = eps
+        fd[i] = (kl_row(q, keys, scale, sc + e)[2] - kl_row(q, keys, scale, sc - e)[2]) / (2 * eps)
+    assert np.allclose(g, fd, atol=1e-8), (g, fd)
+
+
+def check_kl_zero_at_match(kl_row):
+    """KL >= 0, and it vanishes (with its gradient) exactly when the indexer's
+    distribution equals the target: scores = log p + c."""
+    q, keys, scale, sc = _kl_case(2)
+    p, r, kl, g = kl_row(q, keys, scale, sc)
+    assert kl > 1e-3 and abs(p.sum() - 1.0) < 1e-12 and abs(r.sum() - 1.0) < 1e-12
+    assert abs(g.sum()) < 1e-12
+    p2, r2, kl2, g2 = kl_row(q, keys, scale, np.log(p) + 3.25)
+    assert abs(kl2) < 1e-12 and np.abs(g2).max() < 1e-12 and np.allclose(r2, p)
+
+
+def check_kl_one_head_is_softmax(kl_row):
+    """With one head the target is that head's softmax of the scaled logits
+    (torch's softmax); with two heads it is the mean of the two."""
+    q, keys, scale, sc = _kl_case(3, H=2)
+    p1 = kl_row(q[:1], keys, scale, sc)[0]
+    t = torch.softmax(torch.from_numpy(scale * (q[:1] @ keys.T)), dim=-1)[0].numpy()
+    assert np.allclose(p1, t, atol=1e-13)
+    p2 = kl_row(q, keys, scale, sc)[0]
+    t2 = torch.softmax(torch.from_numpy(scale * (q @ keys.T)), dim=-1).mean(0).numpy()
+    assert np.allclose(p2, t2, atol=1e-13)
+
+
+def check_kl_bruteforce(kl_row):
+    """Python loops with math.exp / math.log on a tiny case."""
+    import math
+    q, keys, scale, sc = _kl_case(4, H=2, n=3, d=2)
+    H, n = q.shape[0], keys.shape[0]
+    p = [0.0] * n
+    for h in range(H):
+        z = [scale * sum(q[h, c] * keys[i, c] for c in range(q.shape[1])) for i in range(n)]
+        den = sum(math.exp(x) for x in z)
+        for i in range(n):
+            p[i] += math.exp(z[i]) / den / H
+    den = sum(math.exp(x) for x in sc)
+    r = [math.exp(x) / den for x in sc]
+    kl = sum(p[i] * (math.log(p[i]) - math.log(r[i])) for i in range(n))
+    P, R, KL, G = kl_row(q, keys, scale, sc)
+    assert np.allclose(P, p, atol=1e-14) and np.allclose(R, r, atol=1e-14)
+    assert abs(KL - kl) < 1e-13 and np.allclose(G, np.array(r) - np.array(p), atol=1e-14)
+
+
+def check_kl_dense_stage_reduction(kl_rows, topk_row):
+    """With k >= t + 1 the selection is every preceding key, so the sparse-stage
+    signal over the selection is the dense warm-up signal over the whole prefix
+    (computed here directly from the row's keys 0..t)."""
+    rng = np.random.default_rng(5)
+    L, H, d = 9, 4, 6
+    q = rng.standard_normal((L, H, d))
+    kv = rng.standard_normal((L, d))
+    scores = rng.standard_normal((L, L))
+    rows = list(range(L))
+    idx = np.stack([topk_row(scores[t], t, 16) for t in rows])
+    sel = np.where(idx >= 0, np.take_along_axis(scores, np.maximum(idx, 0), 1), -np.inf)
+    p, kl, g = kl_rows(q, kv, idx, rows, 0.5, sel)
+    for t in rows:
+        P, R, KL, G = O.indexer_kl_row(q[t], kv[: t + 1], 0.5, scores[t, : t + 1])
+        assert abs(kl[t] - KL) < 1e-12 and np.allclose(p[t, : t + 1], P, atol=1e-14)
+        assert np.allclose(g[t, : t + 1], G, atol=1e-14) and np.all(g[t, t + 1:] == 0)
+
+
 def check_paged(paged_rows):
     rng = np.random.default_rng(12)
     P, n_pages, d = 4, 7, 3
@@ -335,6 +415,26 @@ def test_dense_vs_sdpa():
 
 def test_attention_properties():
     check_attention_properties(O.attend, O.sparse_mqa_row)
+
+
+def test_kl_gradient_finite_differences():
+    check_kl_gradient_finite_differences(O.indexer_kl_row)
+
+
+def test_kl_zero_at_match():
+    check_kl_zero_at_match(O.indexer_kl_row)
+
+
+def test_kl_one_head_is_softmax():
+    check_kl_one_head_is_softmax(O.indexer_kl_row)
+
+
+def test_kl_bruteforce():
+    check_kl_bruteforce(O.indexer_kl_row)
+
+
+def test_kl_dense_stage_reduction():
+    check_kl_dense_stage_reduction(O.indexer_kl_rows, O.topk_row)
 
 
 def test_paged_rows():
@@ -448,7 +548,38 @@ def _mut_dequantize_divide(codes, scale):
     return x / s.reshape(s.shape + (1,) * (x.ndim - s.ndim))
 
 
+def _mut_kl_reversed(q_t, keys, scale, scores):
+    p, r, _, g = O.indexer_kl_row(q_t, keys, scale, scores)
+    return p, r, float(np.sum(r * (np.log(r) - np.log(p)))), g      # KL(r || p)
+
+
+def _mut_kl_head_sum(q_t, keys, scale, scores):
+    _, _, probs = O.attend(q_t, keys, np.asarray(keys)[:, :1], scale)
+    p = probs.sum(axis=0)                                            # not averaged
+    s = np.asarray(scores, dtype=np.float64)
+    r = np.exp(s - s.max()); r /= r.sum()
+    return p, r, float(np.sum(p * (np.log(p) - np.log(r)))), r - p
+
+
+def _mut_kl_grad_sign(q_t, keys, scale, scores):
+    p, r, kl, g = O.indexer_kl_row(q_t, keys, scale, scores)
+    return p, r, kl, -g
+
+
+def _mut_kl_softmax_over_heads(q_t, keys, scale, scores):
+    z = scale * (np.asarray(q_t) @ np.asarray(keys).T)
+    e = np.exp(z - z.max(axis=0, keepdims=True))
+    p = (e / e.sum(axis=0, keepdims=True)).mean(axis=0)              # softmax across heads
+    s = np.asarray(scores, dtype=np.float64)
+    r = np.exp(s - s.max()); r /= r.sum()
+    return p, r, float(np.sum(p * (np.log(p) - np.log(r)))), r - p
+
+
 PLANTED = [
+    ("kl reversed", lambda: check_kl_gradient_finite_differences(_mut_kl_reversed)),
+    ("kl head sum", lambda: check_kl_zero_at_match(_mut_kl_head_sum)),
+    ("kl grad sign", lambda: check_kl_gradient_finite_differences(_mut_kl_grad_sign)),
+    ("kl softmax over heads", lambda: check_kl_one_head_is_softmax(_mut_kl_softmax_over_heads)),
     ("decode bias", lambda: check_e4m3_golden(_mut_decode_bias)),
     ("decode bias/torch", lambda: check_e4m3_vs_torch(_mut_decode_bias)),
     ("decode subnormal", lambda: check_e4m3_vs_torch(_mut_decode_subnormal)),
