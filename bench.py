@@ -375,6 +375,9 @@ def run_ours(args, world, rank, local):
     curve = None
     if not args.skip_curve:
         curve = cost_vs_position(dsa, inp, wl, k, world, peaks)
+    kl = None
+    if not args.skip_kl:
+        kl = indexer_kl_signal(dsa, inp, wl, ind, att, ws, idx, out, lse, k, world, peaks)
 
     # ------------------------------------------------------------ e2e (host buffers)
     e2e = None
@@ -400,7 +403,7 @@ def run_ours(args, world, rank, local):
                    "l2": "inputs larger than L2 (q alone 19.3 GB)",
                    "parallelism": f"replicas x{world} (independent sequences)"},
         "roofline": roof, "rooflines": rooflines, "fp8_peak": fp8, "stages": stages,
-        "cpu_baseline": cpu, "e2e": e2e, "cost_vs_position": curve,
+        "cpu_baseline": cpu, "e2e": e2e, "cost_vs_position": curve, "indexer_kl": kl,
         "gpu_launches": int(round(per_call * args.steps)),
         "clocks": clk.summary(),
     }
@@ -445,6 +448,32 @@ def cost_vs_position(dsa, inp, wl, k, world, peaks, block=4096, steps=2,
     return {"block_queries": block, "unit": "ms per block of queries", "points": pts,
             "how": "queries P-block..P-1 against keys 0..P-1 of the 128K inputs; dsa = "
                    "dsa_forward (indexer, top-k, sparse attention), dense = dsa_dense_mqa_fwd"}
+
+
+def indexer_kl_signal(dsa, inp, wl, ind, att, ws, idx, out, lse, k, world, peaks, steps=2):
+    """The indexer's KL training signal over the whole prefill (what a sparse
+    training step adds to the forward): the selection with its kept scores
+    (dsa_select_scored) and the signal (dsa_indexer_kl) from the forward's lse.
+    The KL kernel recomputes q.k for all 128 heads and 576 dims of every
+    selected pair: 2 * 128 * 576 flops per pair."""
+    L = wl.L
+    sel = torch.empty(L, k, device="cuda")
+    loss = torch.empty(L, device="cuda")
+    grad = torch.empty(L, k, device="cuda")
+    dsa.dsa_forward(ind, att, k, idx, out, lse, ws)
+    ms_sel = timed(lambda: dsa.dsa_select_scored(ind, k, idx, sel, ws), steps, 1, world)
+    ms_kl = timed(lambda: dsa.dsa_indexer_kl(att, idx, k, lse, sel, loss, grad), steps, 1, world)
+    st = dsa.dsa_check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {dsa.status_string(st)}")
+    flops = 2.0 * wl.H * wl.D_K * attention_pairs(L, k)
+    tf = flops / (ms_kl * 1e-3) / 1e12
+    res = {"select_scored_ms": ms_sel, "indexer_kl_ms": ms_kl, "kl_bf16_tflops": tf,
+           "kl_frac_bf16_sustained": tf / peaks["bf16_sustained"],
+           "mean_loss": float(loss.mean()),
+           "how": "dsa_select_scored + dsa_indexer_kl over the 128K prefill, lse from dsa_forward"}
+    del sel, loss, grad
+    return res
 
 
 def prefill_e2e(dsa, inp, ind, att, ws, idx, out, lse, k, args, world, n_chunks=8):
@@ -677,6 +706,8 @@ def main():
                          "for multi-pass profiling")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-kl", action="store_true",
+                    help="skip the indexer KL training-signal measurement")
     ap.add_argument("--skip-curve", action="store_true",
                     help="skip the prefill cost-vs-position curve (DSA against dense)")
     ap.add_argument("--skip-fp8-peak", action="store_true",

@@ -225,6 +225,37 @@ DSA_API dsa_status dsa_forward(const dsa_indexer_in* indexer, const dsa_attn_in*
                                int32_t k, int32_t* idx_out, void* out, float* lse,
                                void* ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* Steps 1-2 fused like dsa_select, also writing the indexer score of every
+ * kept key: sel_scores[r*ld_sel + i] is the score of key idx[r*ld_idx + i]
+ * (-INFINITY where idx is -1), the very value the selection ranked -- bit for
+ * bit what dsa_indexer_scores gives for that key. These are the indexer-side
+ * inputs of dsa_indexer_kl. Workspace as dsa_select. */
+DSA_API dsa_status dsa_select_scored(const dsa_indexer_in* indexer, int32_t k, int32_t* idx,
+                                     int64_t ld_idx, float* sel_scores, int64_t ld_sel,
+                                     void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* The indexer's KL training signal over each query's selected keys. The
+ * indexer is trained to match the main attention's distribution with a
+ * KL-divergence loss, over every preceding key in the dense warm-up and with
+ * only the top-k keys selected in sparse training (wiki-for-amaranth report,
+ * section "DeepSeek Sparse Attention (DSA)"; juhe.plus read-through, stages
+ * "Dense Warm-up" and "Sparse Training"; 53ai.com read-through, continued
+ * pre-training). For query i with selected keys j (idx row i, entries < 0 or
+ * past the query's position skipped):
+ *   p_j = (1/H) sum_h exp(scale * q[i,h] . kv[key_j] - lse[i,h])  (main attention, heads averaged)
+ *   r_j = softmax_j(sel_scores[i, j])                               (the indexer)
+ *   loss[i] = sum_j p_j (log p_j - log r_j),  grad[i*ld_grad + j] = r_j - p_j (0 when skipped),
+ * the gradient of the loss with respect to the indexer scores (p held fixed).
+ * attn: the forward's attention inputs (BF16, H=128, d_qk=576, CONTIGUOUS or
+ * PAGED); lse: [n_q, 128] the forward's log-sum-exp (dsa_sparse_mqa_fwd /
+ * dsa_forward) of this selection; sel_scores: from dsa_select_scored. With a
+ * selection of every key 0..pos (k >= pos + 1) this is the dense warm-up
+ * signal. No workspace. */
+DSA_API dsa_status dsa_indexer_kl(const dsa_attn_in* attn, const int32_t* idx, int64_t ld_idx,
+                                  int32_t k, const float* lse, const float* sel_scores,
+                                  int64_t ld_sel, float* loss, float* grad, int64_t ld_grad,
+                                  dsa_stream_t stream);
+
 /* Workspace bytes for `op` with these inputs (arguments an op does not use may
  * be NULL/0). The workspace must be 256-byte aligned device memory. */
 DSA_API dsa_status dsa_workspace_size(int32_t op, const dsa_indexer_in* indexer,

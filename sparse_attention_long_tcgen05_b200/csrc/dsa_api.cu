@@ -5,11 +5,13 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "dsa.h"
 #include "dsa_kernels.h"
@@ -63,6 +65,27 @@ dsa_status cuda_fail(cudaError_t e) {
     dsa_status s_ = (expr);                         \
     if (s_ != DSA_OK) return s_;                    \
   } while (0)
+
+// NVTX ranges around each call and each score block, for a timeline profiler;
+// on only when the environment variable DSA_NVTX is set to a non-zero value
+// (read once). Off, a range costs one branch.
+bool nvtx_on() {
+  static const bool on = [] {
+    const char* v = std::getenv("DSA_NVTX");
+    return v != nullptr && v[0] != '\0' && v[0] != '0';
+  }();
+  return on;
+}
+
+struct NvtxRange {
+  bool pushed;
+  explicit NvtxRange(const char* name) : pushed(nvtx_on()) {
+    if (pushed) nvtxRangePushA(name);
+  }
+  ~NvtxRange() {
+    if (pushed) nvtxRangePop();
+  }
+};
 
 // Device status word address and SM count of the current device (set up once
 // per device, with that device current).
@@ -324,8 +347,8 @@ dsa_status run_indexer(const dsa_indexer_in& in, const int32_t* rows, int32_t q_
 // else pos_base + r.
 dsa_status run_topk(const float* scores, int64_t ld_scores, const int32_t* row_pos,
                     int32_t pos_base, const dsa::KeySide* keys, int32_t n_rows, int32_t k,
-                    int32_t* idx, int64_t ld_idx, bool pdl, DeviceInfo* dev,
-                    cudaStream_t stream) {
+                    int32_t* idx, int64_t ld_idx, float* sel, int64_t ld_sel, bool pdl,
+                    DeviceInfo* dev, cudaStream_t stream) {
   dsa::TopkArgs a{};
   a.scores = scores;
   a.ld_scores = ld_scores;
@@ -336,8 +359,13 @@ dsa_status run_topk(const float* scores, int64_t ld_scores, const int32_t* row_p
   a.k = k;
   a.idx = idx;
   a.ld_idx = ld_idx;
+  a.sel = sel;
+  a.ld_sel = ld_sel;
   a.status = dev->status;
-  DSA_LAUNCH(dsa::launch_topk(a, pdl, stream));
+  // few rows (a decode batch): two CTAs per row so the row's two passes use
+  // twice the SMs
+  const bool pair = 2 * static_cast<int64_t>(n_rows) <= dev->num_sms;
+  DSA_LAUNCH(dsa::launch_topk(a, pdl, pair, stream));
   return DSA_OK;
 }
 
@@ -386,23 +414,27 @@ dsa_status run_attn(const dsa_attn_in& in, const int32_t* idx, int64_t ld_idx, i
 // Indexer -> top-k over bounded blocks of `chunk` query rows, the scores of
 // one block living only in `scores` (chunk x n_cols floats). Prefill block
 // rows see keys 0..off+q0+rows-1; paged rows see their sequence's pages.
+// sel (nullable) receives the kept keys' scores, laid out like idx.
 dsa_status run_select(const dsa_indexer_in& ind, int32_t k, int32_t* idx, int64_t ld_idx,
                       float* scores, int32_t n_cols, int32_t chunk, DeviceInfo* dev,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, float* sel = nullptr, int64_t ld_sel = 0) {
   const int32_t n_q = ind.n_q;
   const bool paged = ind.kv.kind == DSA_KV_PAGED;
   const int32_t off = paged ? 0 : ind.n_keys - n_q;  // position of query 0 (contiguous)
   for (int32_t q0 = 0; q0 < n_q; q0 += chunk) {
+    NvtxRange range("dsa score block (indexer + top-k)");
     const int32_t rows = n_q - q0 < chunk ? n_q - q0 : chunk;
     int32_t* out = idx + static_cast<int64_t>(q0) * ld_idx;
+    float* sel_out = sel ? sel + static_cast<int64_t>(q0) * ld_sel : nullptr;
     const int32_t cols = paged ? n_cols : off + q0 + rows;  // keys any row of the block sees
     DSA_TRY(run_indexer(ind, nullptr, q0, rows, scores, cols, cols, 0, q0 > 0, dev, stream));
     if (paged) {  // row r is query q0 + r at its own position in its sequence
       const dsa::KeySide ks = key_side(ind.kv, n_q, ind.n_keys);
-      DSA_TRY(run_topk(scores, cols, nullptr, q0, &ks, rows, k, out, ld_idx, true, dev, stream));
+      DSA_TRY(run_topk(scores, cols, nullptr, q0, &ks, rows, k, out, ld_idx, sel_out, ld_sel, true,
+                       dev, stream));
     } else {
-      DSA_TRY(run_topk(scores, cols, nullptr, off + q0, nullptr, rows, k, out, ld_idx, true, dev,
-                       stream));
+      DSA_TRY(run_topk(scores, cols, nullptr, off + q0, nullptr, rows, k, out, ld_idx, sel_out,
+                       ld_sel, true, dev, stream));
     }
   }
   return DSA_OK;
@@ -416,6 +448,7 @@ DSA_API dsa_status dsa_indexer_scores(const dsa_indexer_in* in, const int32_t* r
                                       int32_t n_rows, float* scores, int64_t ld_scores,
                                       int32_t n_cols, void* ws, size_t ws_bytes,
                                       dsa_stream_t stream) {
+  NvtxRange range("dsa_indexer_scores");
   (void)ws;
   (void)ws_bytes;
   DSA_TRY(check_indexer(in));
@@ -433,18 +466,20 @@ DSA_API dsa_status dsa_indexer_scores(const dsa_indexer_in* in, const int32_t* r
 DSA_API dsa_status dsa_topk(const float* scores, int64_t ld_scores, const int32_t* row_pos,
                             int32_t n_rows, int32_t k, int32_t* idx, int64_t ld_idx,
                             dsa_stream_t stream) {
+  NvtxRange range("dsa_topk");
   if (scores == nullptr || row_pos == nullptr || idx == nullptr || n_rows < 1 || ld_scores < 1)
     return DSA_ERR_INVALID_ARG;
   if (k < 1 || k > kKMax || ld_idx < k) return DSA_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   DSA_TRY(device_info(&dev));
-  return run_topk(scores, ld_scores, row_pos, 0, nullptr, n_rows, k, idx, ld_idx, false, dev,
-                  reinterpret_cast<cudaStream_t>(stream));
+  return run_topk(scores, ld_scores, row_pos, 0, nullptr, n_rows, k, idx, ld_idx, nullptr, 0,
+                  false, dev, reinterpret_cast<cudaStream_t>(stream));
 }
 
 DSA_API dsa_status dsa_sparse_mqa_fwd(const dsa_attn_in* in, const int32_t* idx, int64_t ld_idx,
                                       int32_t k, void* out, float* lse, void* ws,
                                       size_t ws_bytes, dsa_stream_t stream) {
+  NvtxRange range("dsa_sparse_mqa_fwd");
   (void)ws;
   (void)ws_bytes;
   DSA_TRY(check_attn(in));
@@ -458,6 +493,7 @@ DSA_API dsa_status dsa_sparse_mqa_fwd(const dsa_attn_in* in, const int32_t* idx,
 
 DSA_API dsa_status dsa_dense_mqa_fwd(const dsa_attn_in* in, void* out, float* lse,
                                      dsa_stream_t stream) {
+  NvtxRange range("dsa_dense_mqa_fwd");
   DSA_TRY(check_attn(in));
   if (out == nullptr) return DSA_ERR_INVALID_ARG;
   if (in->dtype == DSA_BF16 && !aligned16(out)) return DSA_ERR_INVALID_ARG;
@@ -467,6 +503,39 @@ DSA_API dsa_status dsa_dense_mqa_fwd(const dsa_attn_in* in, void* out, float* ls
   DSA_TRY(device_info(&dev));
   return run_attn(*in, nullptr, 0, in->dtype == DSA_F32 ? in->n_keys : 0, out, lse, dev,
                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+DSA_API dsa_status dsa_indexer_kl(const dsa_attn_in* attn, const int32_t* idx, int64_t ld_idx,
+                                  int32_t k, const float* lse, const float* sel_scores,
+                                  int64_t ld_sel, float* loss, float* grad, int64_t ld_grad,
+                                  dsa_stream_t stream) {
+  NvtxRange range("dsa_indexer_kl");
+  DSA_TRY(check_attn(attn));
+  if (attn->dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+  if (idx == nullptr || lse == nullptr || sel_scores == nullptr || loss == nullptr ||
+      grad == nullptr || k < 1 || k > kKMax || ld_idx < k || ld_sel < k || ld_grad < k)
+    return DSA_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  DSA_TRY(device_info(&dev));
+  dsa::KlArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(attn->q);
+  a.ld_q = attn->ld_q;
+  a.kv = static_cast<const __nv_bfloat16*>(attn->kv);
+  a.ld_kv = attn->ld_kv;
+  a.idx = idx;
+  a.ld_idx = ld_idx;
+  a.k = k;
+  a.keys = key_side(attn->kv_layout, attn->n_q, attn->n_keys);
+  a.scale_log2 = attn->scale * 1.4426950408889634f;
+  a.lse = lse;
+  a.sel = sel_scores;
+  a.ld_sel = ld_sel;
+  a.loss = loss;
+  a.grad = grad;
+  a.ld_grad = ld_grad;
+  a.status = dev->status;
+  DSA_LAUNCH(dsa::launch_indexer_kl(a, reinterpret_cast<cudaStream_t>(stream)));
+  return DSA_OK;
 }
 
 DSA_API dsa_status dsa_workspace_size(int32_t op, const dsa_indexer_in* indexer,
@@ -498,6 +567,7 @@ DSA_API dsa_status dsa_workspace_size(int32_t op, const dsa_indexer_in* indexer,
 DSA_API dsa_status dsa_forward(const dsa_indexer_in* indexer, const dsa_attn_in* attn,
                                int32_t k, int32_t* idx_out, void* out, float* lse, void* ws,
                                size_t ws_bytes, dsa_stream_t stream_) {
+  NvtxRange range("dsa_forward");
   DSA_TRY(check_indexer(indexer));
   DSA_TRY(check_attn(attn));
   if (out == nullptr || k < 1 || k > kKMax) return DSA_ERR_INVALID_ARG;
@@ -533,6 +603,7 @@ DSA_API dsa_status dsa_forward(const dsa_indexer_in* indexer, const dsa_attn_in*
 
 DSA_API dsa_status dsa_select(const dsa_indexer_in* indexer, int32_t k, int32_t* idx,
                               int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  NvtxRange range("dsa_select");
   DSA_TRY(check_indexer(indexer));
   if (idx == nullptr || k < 1 || k > kKMax || ld_idx < k) return DSA_ERR_INVALID_ARG;
   const ForwardPlan p = forward_plan(*indexer, k);
@@ -542,6 +613,22 @@ DSA_API dsa_status dsa_select(const dsa_indexer_in* indexer, int32_t k, int32_t*
   DSA_TRY(device_info(&dev));
   return run_select(*indexer, k, idx, ld_idx, static_cast<float*>(ws), p.n_cols, p.chunk, dev,
                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+DSA_API dsa_status dsa_select_scored(const dsa_indexer_in* indexer, int32_t k, int32_t* idx,
+                                     int64_t ld_idx, float* sel_scores, int64_t ld_sel,
+                                     void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  NvtxRange range("dsa_select_scored");
+  DSA_TRY(check_indexer(indexer));
+  if (idx == nullptr || sel_scores == nullptr || k < 1 || k > kKMax || ld_idx < k || ld_sel < k)
+    return DSA_ERR_INVALID_ARG;
+  const ForwardPlan p = forward_plan(*indexer, k);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < p.scores_bytes)
+    return DSA_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  DSA_TRY(device_info(&dev));
+  return run_select(*indexer, k, idx, ld_idx, static_cast<float*>(ws), p.n_cols, p.chunk, dev,
+                    reinterpret_cast<cudaStream_t>(stream), sel_scores, ld_sel);
 }
 
 DSA_API int64_t dsa_launch_counter(void) { return g_launches.load(); }

@@ -90,11 +90,14 @@ struct TopkArgs {
   int32_t k;
   int32_t* idx;
   int64_t ld_idx;
+  float* sel;              // nullable: the kept keys' scores, laid out like idx (-inf padding)
+  int64_t ld_sel;
   int* status;
 };
 
-// pdl: as for launch_indexer_fp8.
-cudaError_t launch_topk(const TopkArgs& a, bool pdl, cudaStream_t stream);
+// pdl: as for launch_indexer_fp8. pair: each row on a cluster of two CTAs
+// (for calls with at most half as many rows as SMs); same results.
+cudaError_t launch_topk(const TopkArgs& a, bool pdl, bool pair, cudaStream_t stream);
 
 // ---------------------------------------------------------------- attention
 
@@ -134,6 +137,29 @@ struct AttnF32Args {
 };
 
 cudaError_t launch_attn_f32(const AttnF32Args& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- indexer KL signal
+
+struct KlArgs {
+  const __nv_bfloat16* q;   // [n_q, 128, 576]
+  int64_t ld_q;
+  const __nv_bfloat16* kv;  // latent KV rows [rows, 576] (contiguous, or pages of 64 rows)
+  int64_t ld_kv;
+  const int32_t* idx;       // [n_q, ld_idx] selected key positions (-1 skipped)
+  int64_t ld_idx;
+  int32_t k;
+  KeySide keys;
+  float scale_log2;         // softmax scale * log2(e)
+  const float* lse;         // [n_q, 128] the forward's natural-log LSE over the selection
+  const float* sel;         // [n_q, ld_sel] indexer scores of the selected entries
+  int64_t ld_sel;
+  float* loss;              // [n_q]
+  float* grad;              // [n_q, ld_grad]
+  int64_t ld_grad;
+  int* status;
+};
+
+cudaError_t launch_indexer_kl(const KlArgs& a, cudaStream_t stream);
 
 // Sequence and position of paged query qi (the rule of the ABI's PAGED
 // layout): the sequence is q_seq[qi] (qi when q_seq is null), whose ctx_lens

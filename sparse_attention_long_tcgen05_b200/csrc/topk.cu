@@ -36,6 +36,7 @@ struct TopkSmem {
   uint32_t hist[4096];
   uint32_t warp_sums[kWarps + 1];
   uint32_t found[2];
+  uint32_t m_pub;                           // pair mode: this CTA's collected count
   int32_t lidx[kCap];
   uint32_t lkey[kCap];
 };
@@ -137,7 +138,8 @@ __device__ __forceinline__ void clear_hist(uint32_t* hist, int nb) {
 // inside a warp's 256-pair segment, so one block scan covers kChunk pairs.
 template <class Get>
 __device__ __forceinline__ void ordered_emit(int m, uint32_t T, uint32_t take_eq, int k,
-                                             int32_t* out, uint32_t* warp_sums, Get get) {
+                                             int32_t* out, float* sel, const float* row,
+                                             uint32_t* warp_sums, Get get) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const uint32_t lt = (1u << lane) - 1u;
   uint32_t run_gt = 0, run_eq = 0;
@@ -167,7 +169,11 @@ __device__ __forceinline__ void ordered_emit(int m, uint32_t T, uint32_t take_eq
       const uint32_t e_me = eq_b + __popc(beq[j] & lt);
       const bool gt = (bgt[j] >> lane) & 1u;
       const bool eq = (beq[j] >> lane) & 1u;
-      if (gt || (eq && e_me < take_eq)) out[g_me + min(e_me, take_eq)] = id[j];
+      if (gt || (eq && e_me < take_eq)) {
+        const uint32_t o = g_me + min(e_me, take_eq);
+        out[o] = id[j];
+        if (sel != nullptr) sel[o] = row[id[j]];   // the kept key's score, as ranked
+      }
       gt_b += __popc(bgt[j]);
       eq_b += __popc(beq[j]);
     }
@@ -180,7 +186,8 @@ __device__ __forceinline__ void ordered_emit(int m, uint32_t T, uint32_t take_eq
 // Exact select without the shared-memory collection (rows with heavy ties):
 // digits 11/11/10 over the row in global memory, then an ordered compaction of
 // the row.
-__device__ void select_in_global(const float* row, int n, int k, int32_t* out, TopkSmem& S) {
+__device__ void select_in_global(const float* row, int n, int k, int32_t* out, float* sel,
+                                 TopkSmem& S) {
   clear_hist(S.hist, 2048);
   for (int i = threadIdx.x; i < n; i += kThreads) atomicAdd(&S.hist[order_key(row[i]) >> 21], 1u);
   __syncthreads();
@@ -205,20 +212,30 @@ __device__ void select_in_global(const float* row, int n, int k, int32_t* out, T
   find_bin(S.hist, 1024, k_rem, S.warp_sums, S.found);
   const uint32_t T = (prefix << 10) | S.found[0];
   const uint32_t take_eq = S.found[1];
-  ordered_emit(n, T, take_eq, k, out, S.warp_sums, [&](int e, int& id, uint32_t& key) {
+  ordered_emit(n, T, take_eq, k, out, sel, row, S.warp_sums, [&](int e, int& id, uint32_t& key) {
     id = e;
     key = order_key(row[e]);
   });
 }
 
+// kPair: each row runs on a cluster of two CTAs (used when the rows are at
+// most half the SMs, e.g. a decode batch): each CTA histograms and collects
+// one half of the row, the histograms are added through distributed shared
+// memory, the second CTA appends its contenders after the first's in the
+// first CTA's shared memory, and the first CTA finishes as in the one-CTA
+// form. Halves split at a multiple of 4, so both read the row as float4 where
+// it allows; the contenders stay in index order, so the result is the same.
+template <bool kPair>
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
   extern __shared__ uint8_t smem_raw[];
   TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
-  const int r = blockIdx.x;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const int r = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int tid = threadIdx.x;
   const int lane = tid & 31, w = tid >> 5;
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld_scores;
   int32_t* out = a.idx + static_cast<int64_t>(r) * a.ld_idx;
+  float* sel = a.sel ? a.sel + static_cast<int64_t>(r) * a.ld_sel : nullptr;
   griddep_launch_dependents();
   griddep_wait();   // the score rows come from the kernel before this one
   int pos;
@@ -231,14 +248,22 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
     pos = a.pos_base + r;
   }
   if (pos < 0 || pos >= a.ld_scores) {
+    if (rank != 0) return;                         // (both CTAs take this branch)
     if (tid == 0) report(a.status, DSA_ERR_DEVICE_BOUNDS);
-    for (int j = tid; j < a.k; j += kThreads) out[j] = -1;
+    for (int j = tid; j < a.k; j += kThreads) {
+      out[j] = -1;
+      if (sel != nullptr) sel[j] = -INFINITY;
+    }
     return;
   }
   const int n = pos + 1;
   const int k = a.k;
   if (n <= k) {
-    for (int j = tid; j < k; j += kThreads) out[j] = j < n ? j : -1;
+    if (rank != 0) return;
+    for (int j = tid; j < k; j += kThreads) {
+      out[j] = j < n ? j : -1;
+      if (sel != nullptr) sel[j] = j < n ? row[j] : -INFINITY;
+    }
     return;
   }
 
@@ -247,37 +272,57 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
   // row, and a lane keeps four loads in flight where it had one.
   const bool vec = (reinterpret_cast<uintptr_t>(row) & 15u) == 0 && (a.ld_scores & 3) == 0;
   const float4* row4 = reinterpret_cast<const float4*>(row);
+  // this CTA's part of the row: [lo, hi)
+  int lo = 0, hi = n;
+  if (kPair) {
+    const int h0 = min(n, (((n + 1) >> 1) + 3) & ~3);
+    lo = rank == 0 ? 0 : h0;
+    hi = rank == 0 ? h0 : n;
+  }
 
   // ---- pass 1: histogram of the top 12 key bits
   clear_hist(S.hist, 4096);
   if (vec) {
-    const int n4 = (n + 3) >> 2;
-    for (int c = tid; c < n4; c += 4 * kThreads) {
+    const int hi4 = (hi + 3) >> 2;
+    for (int c = (lo >> 2) + tid; c < hi4; c += 4 * kThreads) {
       float4 v[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int q = c + j * kThreads;
-        v[j] = q < n4 ? row4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[j] = q < hi4 ? row4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int i = 4 * (c + j * kThreads);
-        if (i < n) atomicAdd(&S.hist[order_key(v[j].x) >> 20], 1u);
-        if (i + 1 < n) atomicAdd(&S.hist[order_key(v[j].y) >> 20], 1u);
-        if (i + 2 < n) atomicAdd(&S.hist[order_key(v[j].z) >> 20], 1u);
-        if (i + 3 < n) atomicAdd(&S.hist[order_key(v[j].w) >> 20], 1u);
+        if (i < hi) atomicAdd(&S.hist[order_key(v[j].x) >> 20], 1u);
+        if (i + 1 < hi) atomicAdd(&S.hist[order_key(v[j].y) >> 20], 1u);
+        if (i + 2 < hi) atomicAdd(&S.hist[order_key(v[j].z) >> 20], 1u);
+        if (i + 3 < hi) atomicAdd(&S.hist[order_key(v[j].w) >> 20], 1u);
       }
     }
   } else {
-    for (int i = tid; i < n; i += kThreads) atomicAdd(&S.hist[order_key(row[i]) >> 20], 1u);
+    for (int i = lo + tid; i < hi; i += kThreads) atomicAdd(&S.hist[order_key(row[i]) >> 20], 1u);
   }
   __syncthreads();
+  if (kPair) {
+    // add the peer's histogram: read it, let both CTAs finish reading, add
+    const uint32_t peer_hist = mapa_shared(smem_u32(S.hist), rank ^ 1u);
+    uint32_t ph[4096 / kThreads];
+    cluster_sync();                                // both histograms complete
+#pragma unroll
+    for (int i = 0; i < 4096 / kThreads; ++i)
+      ph[i] = ld_shared_cluster_u32(peer_hist + 4u * static_cast<uint32_t>(tid + i * kThreads));
+    cluster_sync();                                // both CTAs have read the peer's
+#pragma unroll
+    for (int i = 0; i < 4096 / kThreads; ++i) S.hist[tid + i * kThreads] += ph[i];
+    __syncthreads();
+  }
   find_bin(S.hist, 4096, static_cast<uint32_t>(k), S.warp_sums, S.found);
   const uint32_t b1 = S.found[0];
   const uint32_t k_rem = S.found[1];
   const uint32_t collect = static_cast<uint32_t>(k) - k_rem + S.hist[b1];
   if (collect > static_cast<uint32_t>(kCap)) {   // uniform: every thread read the same values
-    select_in_global(row, n, k, out, S);
+    if (rank == 0) select_in_global(row, n, k, out, sel, S);
     return;
   }
 
@@ -292,11 +337,11 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
   if (vec) {
 #pragma unroll
     for (int h = 0; h < kPer / 4; ++h) {
-      const int i0 = w * (32 * kPer) + h * 128 + 4 * lane;
-      nxt[h] = i0 < n ? row4[i0 >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int i0 = lo + w * (32 * kPer) + h * 128 + 4 * lane;
+      nxt[h] = i0 < hi ? row4[i0 >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
-  for (int c0 = 0; c0 < n; c0 += kChunk) {
+  for (int c0 = lo; c0 < hi; c0 += kChunk) {
     uint32_t bal[kPer], key[kPer];
     uint32_t cnt = 0;
     const int wbase = c0 + w * (32 * kPer);
@@ -306,26 +351,26 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
       for (int h = 0; h < kPer / 4; ++h) {
         cur[h] = nxt[h];
         const int i1 = wbase + kChunk + h * 128 + 4 * lane;
-        nxt[h] = i1 < n ? row4[i1 >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+        nxt[h] = i1 < hi ? row4[i1 >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int h = 0; h < kPer / 4; ++h) {
         const int i0 = wbase + h * 128 + 4 * lane;
         const float4 v = cur[h];
-        key[4 * h + 0] = i0 < n ? order_key(v.x) : 0u;
-        key[4 * h + 1] = i0 + 1 < n ? order_key(v.y) : 0u;
-        key[4 * h + 2] = i0 + 2 < n ? order_key(v.z) : 0u;
-        key[4 * h + 3] = i0 + 3 < n ? order_key(v.w) : 0u;
+        key[4 * h + 0] = i0 < hi ? order_key(v.x) : 0u;
+        key[4 * h + 1] = i0 + 1 < hi ? order_key(v.y) : 0u;
+        key[4 * h + 2] = i0 + 2 < hi ? order_key(v.z) : 0u;
+        key[4 * h + 3] = i0 + 3 < hi ? order_key(v.w) : 0u;
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          bal[4 * h + e] = __ballot_sync(0xffffffffu, i0 + e < n && (key[4 * h + e] >> 20) >= b1);
+          bal[4 * h + e] = __ballot_sync(0xffffffffu, i0 + e < hi && (key[4 * h + e] >> 20) >= b1);
       }
     } else {
 #pragma unroll
       for (int j = 0; j < kPer; ++j) {
         const int i = wbase + j * 32 + lane;
-        key[j] = i < n ? order_key(row[i]) : 0u;
-        bal[j] = __ballot_sync(0xffffffffu, i < n && (key[j] >> 20) >= b1);
+        key[j] = i < hi ? order_key(row[i]) : 0u;
+        bal[j] = __ballot_sync(0xffffffffu, i < hi && (key[j] >> 20) >= b1);
       }
     }
 #pragma unroll
@@ -363,7 +408,28 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
     base += total;
   }
   __syncthreads();
-  const int m = static_cast<int>(base);
+  int m = static_cast<int>(base);
+  if (kPair) {
+    // the second CTA appends its contenders after the first CTA's, in the
+    // first CTA's shared memory (the two counts add up to `collect`, which
+    // fits the buffer); then the first CTA goes on alone
+    if (tid == 0) S.m_pub = base;
+    cluster_sync();
+    if (rank == 1) {
+      const uint32_t m0 = ld_shared_cluster_u32(mapa_shared(smem_u32(&S.m_pub), 0u));
+      const uint32_t pidx = mapa_shared(smem_u32(S.lidx), 0u);
+      const uint32_t pkey = mapa_shared(smem_u32(S.lkey), 0u);
+      for (int e = tid; e < m; e += kThreads) {
+        st_shared_cluster_u32(pidx + 4u * (m0 + static_cast<uint32_t>(e)),
+                              static_cast<uint32_t>(S.lidx[e]));
+        st_shared_cluster_u32(pkey + 4u * (m0 + static_cast<uint32_t>(e)), S.lkey[e]);
+      }
+    } else {
+      m += static_cast<int>(ld_shared_cluster_u32(mapa_shared(smem_u32(&S.m_pub), 1u)));
+    }
+    cluster_sync();                                // the appended list is in place
+    if (rank == 1) return;
+  }
 
   // ---- exact threshold among the contenders of bin b1 (shared memory only)
   clear_hist(S.hist, 1024);
@@ -386,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
   const uint32_t take_eq = S.found[1];
 
   // ---- ordered emit from the collected list
-  ordered_emit(m, T, take_eq, k, out, S.warp_sums, [&](int e, int& id, uint32_t& kk) {
+  ordered_emit(m, T, take_eq, k, out, sel, row, S.warp_sums, [&](int e, int& id, uint32_t& kk) {
     id = S.lidx[e];
     kk = S.lkey[e];
   });
@@ -394,23 +460,35 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
 
 }  // namespace
 
-cudaError_t launch_topk(const TopkArgs& a, bool pdl, cudaStream_t stream) {
+cudaError_t launch_topk(const TopkArgs& a, bool pdl, bool pair, cudaStream_t stream) {
   if (a.n_rows <= 0) return cudaSuccess;
   const size_t smem = sizeof(TopkSmem);
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kernel = pair ? topk_kernel<true> : topk_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.n_rows);
+  cfg.gridDim = dim3(pair ? 2 * a.n_rows : a.n_rows);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (pair) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 2;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, topk_kernel, a);
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
 }  // namespace dsa

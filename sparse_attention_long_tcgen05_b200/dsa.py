@@ -34,7 +34,7 @@ DSA_OP_SELECT = 4
 EXPORTED = ["dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_fwd", "dsa_select", "dsa_forward",
             "dsa_workspace_size", "dsa_check_status", "dsa_status_string",
             "dsa_last_cuda_error", "dsa_launch_counter", "dsa_version", "dsa_select_noalloc",
-            "dsa_set_wait_limit_ns", "dsa_dense_mqa_fwd"]
+            "dsa_set_wait_limit_ns", "dsa_dense_mqa_fwd", "dsa_select_scored", "dsa_indexer_kl"]
 
 
 class DsaError(RuntimeError):
@@ -81,6 +81,8 @@ def _load():
         "dsa_sparse_mqa_fwd": [ctypes.POINTER(AttnIn), P, I64, I32, P, P, P, SZ, P],
         "dsa_select": [ctypes.POINTER(IndexerIn), I32, P, I64, P, SZ, P],
         "dsa_dense_mqa_fwd": [ctypes.POINTER(AttnIn), P, P, P],
+        "dsa_select_scored": [ctypes.POINTER(IndexerIn), I32, P, I64, P, I64, P, SZ, P],
+        "dsa_indexer_kl": [ctypes.POINTER(AttnIn), P, I64, I32, P, P, I64, P, P, I64, P],
         "dsa_forward": [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), I32, P, P, P, P, SZ, P],
         "dsa_launch_counter": [],
         "dsa_set_wait_limit_ns": [I64],
@@ -217,6 +219,22 @@ def dsa_dense_mqa_fwd(attn: _Keep, out: torch.Tensor, lse: Optional[torch.Tensor
                       stream=None):
     _check(LIB.dsa_dense_mqa_fwd(ctypes.byref(attn.struct), _ptr(out), _ptr(lse),
                                  _stream(stream)), "dsa_dense_mqa_fwd")
+
+
+def dsa_select_scored(ind: _Keep, k: int, idx: torch.Tensor, sel_scores: torch.Tensor,
+                      ws: torch.Tensor, stream=None):
+    _check(LIB.dsa_select_scored(ctypes.byref(ind.struct), k, _ptr(idx), idx.stride(0),
+                                 _ptr(sel_scores), sel_scores.stride(0), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_select_scored")
+
+
+def dsa_indexer_kl(attn: _Keep, idx: torch.Tensor, k: int, lse: torch.Tensor,
+                   sel_scores: torch.Tensor, loss: torch.Tensor, grad: torch.Tensor,
+                   stream=None):
+    _check(LIB.dsa_indexer_kl(ctypes.byref(attn.struct), _ptr(idx), idx.stride(0), k, _ptr(lse),
+                              _ptr(sel_scores), sel_scores.stride(0), _ptr(loss), _ptr(grad),
+                              grad.stride(0), _stream(stream)), "dsa_indexer_kl")
 
 
 def dsa_select(ind: _Keep, k: int, idx: torch.Tensor, ws: torch.Tensor, stream=None):

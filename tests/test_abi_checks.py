@@ -7,6 +7,7 @@ every host check stops at the device lookup with DSA_ERR_CUDA. That is the
 control below -- the unmodified arguments reach the device lookup -- and each
 case changes one field of them and must get its own status instead."""
 import ctypes
+import os
 
 import pytest
 import torch
@@ -266,3 +267,58 @@ def test_noalloc_checks(dsa):
     big = _mut(ind, n_keys=(16 << 20) // 4 + 1)
     _expect(dsa, dsa.DSA_ERR_WORKSPACE_TOO_SMALL,
             lambda: call(ctypes.byref(big), 2048, _p(FAKE), 2048, None))
+
+
+def test_kl_and_select_scored_checks(dsa):
+    ind, att = _indexer(dsa), _attn(dsa)
+    INV, UNS, WS = dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_UNSUPPORTED, \
+        dsa.DSA_ERR_WORKSPACE_TOO_SMALL
+    P = FAKE + 0x200000
+
+    def kl(attn=att, idx=P, ld_idx=2048, k=2048, lse=P, sel=P, ld_sel=2048, loss=P, grad=P,
+           ld_grad=2048):
+        return dsa.LIB.dsa_indexer_kl(ctypes.byref(attn), _p(idx), ld_idx, k, _p(lse), _p(sel),
+                                      ld_sel, _p(loss), _p(grad), ld_grad, None)
+    _expect(dsa, dsa.DSA_ERR_CUDA, lambda: kl())
+    for kw in (dict(idx=None), dict(lse=None), dict(sel=None), dict(loss=None), dict(grad=None),
+               dict(k=0), dict(k=2049), dict(ld_idx=100), dict(ld_sel=100), dict(ld_grad=100)):
+        _expect(dsa, INV, lambda: kl(**kw))
+    f32 = _mut(att, dtype=dsa.DSA_F32, heads=8, d_qk=64, d_v=64, ld_q=512, ld_kv=64)
+    _expect(dsa, UNS, lambda: kl(attn=f32))
+
+    def ss(k=2048, idx=P, ld_idx=2048, sel=P, ld_sel=2048, ws=FAKE + 0x100000, ws_bytes=1 << 34):
+        return dsa.LIB.dsa_select_scored(ctypes.byref(ind), k, _p(idx), ld_idx, _p(sel), ld_sel,
+                                         _p(ws), ws_bytes, None)
+    _expect(dsa, dsa.DSA_ERR_CUDA, lambda: ss())
+    for kw in (dict(idx=None), dict(sel=None), dict(k=0), dict(ld_idx=1), dict(ld_sel=1)):
+        _expect(dsa, INV, lambda: ss(**kw))
+    _expect(dsa, WS, lambda: ss(ws_bytes=1024))
+    _expect(dsa, WS, lambda: ss(ws=None))
+
+    def dense(attn=att, out=FAKE + 0x2000):
+        return dsa.LIB.dsa_dense_mqa_fwd(ctypes.byref(attn), _p(out), None, None)
+    _expect(dsa, dsa.DSA_ERR_CUDA, lambda: dense())
+    _expect(dsa, INV, lambda: dense(out=None))
+    _expect(dsa, INV, lambda: dense(out=FAKE + 0x2004))
+    _expect(dsa, UNS, lambda: dense(attn=_mut(f32, n_keys=5000, n_q=100)))   # fp32 dense > 4096 keys
+
+
+def test_nvtx_ranges_switch_on_without_a_profiler():
+    """DSA_NVTX=1 turns the per-call and per-block NVTX ranges on (read once
+    per process); with no profiler attached they are no-ops and the call
+    behaves as before."""
+    import subprocess
+    import sys
+    code = (
+        "import ctypes, sys; sys.path.insert(0, %r)\n"
+        "from sparse_attention_long_tcgen05_b200 import dsa\n"
+        "import test_abi_checks as t\n"
+        "ind, att = t._indexer(dsa), t._attn(dsa)\n"
+        "st = t._forward(dsa, ind, att)\n"
+        "print(st)\n") % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))),)
+    env = dict(os.environ, DSA_NVTX="1",
+               PYTHONPATH=os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip().splitlines()[-1] == str(4)   # DSA_ERR_CUDA: no device here
