@@ -17,7 +17,9 @@ Every step is the plain definition, in float64, with numpy library primitives
      rows (V = the first d_v columns of the KV row), with the exact softmax and
      its log-sum-exp;
   5. dense causal attention, used to pin step 4 and as the dense baseline;
-  6. the indexer's KL training signal over a key set.
+  6. the indexer's KL training signal over a key set;
+  7. the gradient of step 4 with respect to the queries and the latent KV rows
+     (the main model's sparse training over the same selection).
 
 Sources (web pages on DeepSeek-V3.2 / V3.2-Exp):
   [53ai]  "DeepSeek-V3.2-Exp 技术报告解读" (53ai.com), section
@@ -210,6 +212,59 @@ def indexer_kl_rows(q, kv, idx, rows, scale, sel_scores):
         p_out[r, m] = p
         g_out[r, m] = g
     return p_out, kl, g_out
+
+
+# ------------------------------------------- gradient of the sparse attention
+
+def attend_backward(q_t, keys, values, scale, d_out):
+    """Gradient of attend() for one query token [amaranth] section "DeepSeek
+    Sparse Attention (DSA)", stage B (sparse training: the main model is
+    trained through the attention over the selected keys only; the indexer's
+    input is detached, so no gradient reaches the selection). With
+    z = scale * q K^T, P = softmax_rows(z), O = P V and an upstream gradient
+    dO = d loss / d O, the chain rule gives
+        dP = dO V^T,  dz = P * (dP - rowsum(dO * O)),
+        dq = scale * dz K,  dK = scale * dz^T q,  dV = P^T dO
+    (rowsum(dO * O) = sum_i P_i dP_i is the softmax Jacobian's correction).
+    q_t [H, d_qk], keys [n, d_qk], values [n, d_v], d_out [H, d_v].
+    Returns (dq [H, d_qk], dk [n, d_qk], dv [n, d_v])."""
+    q_t = np.asarray(q_t, dtype=np.float64)
+    keys = np.asarray(keys, dtype=np.float64)
+    values = np.asarray(values, dtype=np.float64)
+    d_out = np.asarray(d_out, dtype=np.float64)
+    out, _, p = attend(q_t, keys, values, scale)
+    dp = d_out @ values.T                                  # [H, n]
+    delta = np.sum(d_out * out, axis=1, keepdims=True)     # [H, 1]
+    dz = p * (dp - delta)                                  # d loss / d z
+    dq = scale * (dz @ keys)
+    dk = scale * (dz.T @ q_t)
+    dv = p.T @ d_out
+    return dq, dk, dv
+
+
+def sparse_mqa_backward(q, kv, idx, rows, d_out, scale, d_v):
+    """Gradient of sparse_mqa (MQA mode, V = the first d_v columns of the
+    selected latent rows) for the query rows ``rows`` with selections idx[r]
+    (entries < 0 skipped) and upstream gradients d_out[r] [H, d_v].
+    A latent row serves as key and as value, so its gradient is the sum of its
+    key gradient and (in its first d_v columns) its value gradient, summed over
+    every query that selected it.
+    Returns (dq [len(rows), H, d_qk], dkv [n_kv, d_qk])."""
+    q = np.asarray(q)
+    kv = np.asarray(kv, dtype=np.float64)
+    idx = np.asarray(idx)
+    H, d_qk = q.shape[1], q.shape[2]
+    dq = np.zeros((len(rows), H, d_qk))
+    dkv = np.zeros(kv.shape)
+    for r, row in enumerate(rows):
+        sel = idx[r][idx[r] >= 0]
+        if sel.size == 0:
+            continue
+        keys = kv[sel]
+        dq[r], dk, dv = attend_backward(q[row], keys, keys[:, :d_v], scale, d_out[r])
+        np.add.at(dkv, sel, dk)
+        np.add.at(dkv[:, :d_v], sel, dv)
+    return dq, dkv
 
 
 # ------------------------------------------------------------- paged caches

@@ -334,6 +334,84 @@ def check_kl_dense_stage_reduction(kl_rows, topk_row):
         assert np.allclose(g[t, : t + 1], G, atol=1e-14) and np.all(g[t, t + 1:] == 0)
 
 
+def _bwd_case(seed=0, L=6, H=2, d=5, dv=3):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((L, H, d))
+    kv = rng.standard_normal((L + 2, d))
+    d_out = rng.standard_normal((L, H, dv))
+    idx = np.full((L, 4), -1)
+    for t in range(L):
+        sel = rng.choice(L + 2, size=min(t + 1, 4), replace=False)
+        idx[t, : sel.size] = np.sort(sel)
+    return q, kv, d_out, idx
+
+
+def check_bwd_finite_differences(bwd):
+    """dq and dkv against central differences of loss = sum(dO * O), O from the
+    (separately pinned) forward sparse_mqa."""
+    q, kv, d_out, idx = _bwd_case(7)
+    rows = list(range(q.shape[0]))
+    scale, dv = 0.7, d_out.shape[2]
+
+    def loss(qq, kk):
+        out, _ = O.sparse_mqa(qq, kk, None, idx, rows, scale, dv)
+        return float(np.sum(out * d_out))
+
+    dq, dkv = bwd(q, kv, idx, rows, d_out, scale, dv)
+    eps = 1e-6
+    fq = np.zeros_like(q)
+    for i in np.ndindex(q.shape):
+        e = np.zeros_like(q)
+        e[i] = eps
+        fq[i] = (loss(q + e, kv) - loss(q - e, kv)) / (2 * eps)
+    fk = np.zeros_like(kv)
+    for i in np.ndindex(kv.shape):
+        e = np.zeros_like(kv)
+        e[i] = eps
+        fk[i] = (loss(q, kv + e) - loss(q, kv - e)) / (2 * eps)
+    assert np.allclose(dq, fq, atol=1e-7), np.abs(dq - fq).max()
+    assert np.allclose(dkv, fk, atol=1e-7), np.abs(dkv - fk).max()
+
+
+def check_bwd_vs_torch_autograd(bwd):
+    """Selecting every preceding key reduces the sparse gradient to dense causal
+    MQA attention's, taken here from torch autograd through
+    scaled_dot_product_attention (float64, CPU), with the keys broadcast over
+    the heads and the values the first dv columns of the same rows."""
+    rng = np.random.default_rng(8)
+    L, H, d, dv, scale = 7, 3, 6, 4, 0.45
+    q = rng.standard_normal((L, H, d))
+    kv = rng.standard_normal((L, d))
+    d_out = rng.standard_normal((L, H, dv))
+    idx = np.stack([O.topk_row(np.zeros(L), t, L) for t in range(L)])
+    dq, dkv = bwd(q, kv, idx, list(range(L)), d_out, scale, dv)
+    tq = torch.from_numpy(q).permute(1, 0, 2)[None].clone().requires_grad_(True)
+    tkv = torch.from_numpy(kv).clone().requires_grad_(True)
+    k = tkv[None, None].expand(1, H, L, d)
+    v = tkv[None, None, :, :dv].expand(1, H, L, dv)
+    out = torch.nn.functional.scaled_dot_product_attention(tq, k, v, is_causal=True, scale=scale)
+    out.backward(torch.from_numpy(d_out).permute(1, 0, 2)[None])
+    assert np.allclose(dq, tq.grad[0].permute(1, 0, 2).numpy(), atol=1e-12)
+    assert np.allclose(dkv, tkv.grad.numpy(), atol=1e-12)
+
+
+def check_bwd_invariants(bwd):
+    """Exact at any size: every softmax row's logit gradient sums to zero, so
+    the key gradients of a query sum to zero and the rope columns of dkv (keys
+    only) sum to zero over the rows; the value gradients of a query sum to its
+    dO (the probabilities sum to one), so the first dv columns of dkv sum to the
+    sum of dO over queries with a non-empty selection and over heads. A query
+    with an empty selection gets dq = 0."""
+    q, kv, d_out, idx = _bwd_case(9, L=12, H=3, d=7, dv=4)
+    idx[5] = -1
+    rows = list(range(q.shape[0]))
+    dq, dkv = bwd(q, kv, idx, rows, d_out, 0.6, 4)
+    assert np.allclose(dkv[:, 4:].sum(axis=0), 0.0, atol=1e-12)
+    live = [t for t in rows if (idx[t] >= 0).any()]
+    assert np.allclose(dkv[:, :4].sum(axis=0), d_out[live].sum(axis=(0, 1)), atol=1e-12)
+    assert np.all(dq[5] == 0.0)
+
+
 def check_paged(paged_rows):
     rng = np.random.default_rng(12)
     P, n_pages, d = 4, 7, 3
@@ -435,6 +513,18 @@ def test_kl_bruteforce():
 
 def test_kl_dense_stage_reduction():
     check_kl_dense_stage_reduction(O.indexer_kl_rows, O.topk_row)
+
+
+def test_bwd_finite_differences():
+    check_bwd_finite_differences(O.sparse_mqa_backward)
+
+
+def test_bwd_vs_torch_autograd():
+    check_bwd_vs_torch_autograd(O.sparse_mqa_backward)
+
+
+def test_bwd_invariants():
+    check_bwd_invariants(O.sparse_mqa_backward)
 
 
 def test_paged_rows():
@@ -575,7 +665,35 @@ def _mut_kl_softmax_over_heads(q_t, keys, scale, scores):
     return p, r, float(np.sum(p * (np.log(p) - np.log(r)))), r - p
 
 
+def _mut_bwd(no_delta=False, dk_scale=True, with_dv=True, dv_off=0):
+    def bwd(q, kv, idx, rows, d_out, scale, d_v):
+        q = np.asarray(q)
+        kv = np.asarray(kv, dtype=np.float64)
+        dq = np.zeros((len(rows),) + q.shape[1:])
+        dkv = np.zeros(kv.shape)
+        for r, row in enumerate(rows):
+            sel = idx[r][idx[r] >= 0]
+            if sel.size == 0:
+                continue
+            keys = kv[sel]
+            vals = keys[:, :d_v]
+            out, _, p = O.attend(q[row], keys, vals, scale)
+            dp = d_out[r] @ vals.T
+            delta = 0.0 if no_delta else np.sum(d_out[r] * out, axis=1, keepdims=True)
+            dz = p * (dp - delta)
+            dq[r] = scale * dz @ keys
+            np.add.at(dkv, sel, (scale if dk_scale else 1.0) * dz.T @ q[row])
+            if with_dv:
+                np.add.at(dkv[:, dv_off:dv_off + d_v], sel, p.T @ d_out[r])
+        return dq, dkv
+    return bwd
+
+
 PLANTED = [
+    ("bwd no delta", lambda: check_bwd_finite_differences(_mut_bwd(no_delta=True))),
+    ("bwd dk unscaled", lambda: check_bwd_finite_differences(_mut_bwd(dk_scale=False))),
+    ("bwd value grad dropped", lambda: check_bwd_invariants(_mut_bwd(with_dv=False))),
+    ("bwd value grad offset", lambda: check_bwd_vs_torch_autograd(_mut_bwd(dv_off=2))),
     ("kl reversed", lambda: check_kl_gradient_finite_differences(_mut_kl_reversed)),
     ("kl head sum", lambda: check_kl_zero_at_match(_mut_kl_head_sum)),
     ("kl grad sign", lambda: check_kl_gradient_finite_differences(_mut_kl_grad_sign)),
