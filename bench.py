@@ -378,6 +378,16 @@ def run_ours(args, world, rank, local):
     kl = None
     if not args.skip_kl:
         kl = indexer_kl_signal(dsa, inp, wl, ind, att, ws, idx, out, lse, k, world, peaks)
+    bwd = None
+    if not args.skip_bwd:
+        bwd = attention_backward(dsa, wl, att, idx, out, lse, k, world, peaks)
+        rooflines["sparse_mqa_bwd_kernel"] = {
+            "bound": "tensor", "achieved": bwd["bf16_tflops"], "peak": peaks["bf16_sustained"],
+            "unit": "TFLOP/s", "frac": bwd["frac_bf16_sustained"],
+            "peak_note": f"bf16 dense sustained ({peaks['source']})",
+            "algorithmic": "2*128*(2*576+576+2*512) bf16 flops per selected (t, key) pair",
+            "launches": 1, "ms": bwd["ms"],
+            "traffic": kernel_traffic("sparse_mqa_bwd_kernel", wl.name)}
 
     # ------------------------------------------------------------ e2e (host buffers)
     e2e = None
@@ -404,6 +414,7 @@ def run_ours(args, world, rank, local):
                    "parallelism": f"replicas x{world} (independent sequences)"},
         "roofline": roof, "rooflines": rooflines, "fp8_peak": fp8, "stages": stages,
         "cpu_baseline": cpu, "e2e": e2e, "cost_vs_position": curve, "indexer_kl": kl,
+        "attention_backward": bwd,
         "gpu_launches": int(round(per_call * args.steps)),
         "clocks": clk.summary(),
     }
@@ -474,6 +485,32 @@ def indexer_kl_signal(dsa, inp, wl, ind, att, ws, idx, out, lse, k, world, peaks
            "how": "dsa_select_scored + dsa_indexer_kl over the 128K prefill, lse from dsa_forward"}
     del sel, loss, grad
     return res
+
+
+def attention_backward(dsa, wl, att, idx, out, lse, k, world, peaks, steps=2):
+    """Gradient of the sparse attention over the 128K prefill's own selection
+    (the main model's side of a sparse training step): dsa_sparse_mqa_bwd with
+    a seeded upstream gradient, given the forward's out and lse. Per selected
+    (t, key) pair it recomputes the logits and dP and forms the query, key and
+    value gradients: 2*128*(576 + 512 + 576 + 576 + 512) flops."""
+    from sparse_attention_long_tcgen05_b200.inputs import make_grad_out
+    L = wl.L
+    d_out = make_grad_out(L, wl.H, wl.D_V, device="cuda", seed=71)
+    dq = torch.empty(L, wl.H, wl.D_K, dtype=torch.bfloat16, device="cuda")
+    dkv = torch.zeros(L, wl.D_K, device="cuda")
+    delta = torch.empty(L, wl.H, 2, device="cuda")
+    ms = timed(lambda: dsa.dsa_sparse_mqa_bwd(att, idx, k, out, lse, d_out, dq, dkv, delta),
+               steps, 1, world)
+    st = dsa.dsa_check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {dsa.status_string(st)}")
+    flops = 2.0 * wl.H * (2 * wl.D_K + wl.D_K + 2 * wl.D_V) * attention_pairs(L, k)
+    tf = flops / (ms * 1e-3) / 1e12
+    del d_out, dq, dkv, delta
+    return {"ms": ms, "bf16_tflops": tf, "frac_bf16_sustained": tf / peaks["bf16_sustained"],
+            "flops": flops, "launches": 2,
+            "how": "dsa_sparse_mqa_bwd (row-dot kernel for D, then the tcgen05 backward) over "
+                   "the 128K selection of dsa_forward; dkv accumulated in fp32"}
 
 
 def prefill_e2e(dsa, inp, ind, att, ws, idx, out, lse, k, args, world, n_chunks=8):
@@ -706,6 +743,8 @@ def main():
                          "for multi-pass profiling")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-bwd", action="store_true",
+                    help="skip the sparse attention backward record")
     ap.add_argument("--skip-kl", action="store_true",
                     help="skip the indexer KL training-signal measurement")
     ap.add_argument("--skip-curve", action="store_true",

@@ -256,6 +256,33 @@ DSA_API dsa_status dsa_indexer_kl(const dsa_attn_in* attn, const int32_t* idx, i
                                   int64_t ld_sel, float* loss, float* grad, int64_t ld_grad,
                                   dsa_stream_t stream);
 
+/* Gradient of step 3 for sparse training: the main model is trained through
+ * the attention over the selected keys only, the indexer's input being detached
+ * (wiki-for-amaranth report, section "DeepSeek Sparse Attention (DSA)", stage
+ * B), so no gradient reaches the selection. For query i (position
+ * n_keys - n_q + i) with selected rows j (idx row i, entries < 0 skipped,
+ * entries past the query's position reported as DSA_ERR_DEVICE_BOUNDS and
+ * skipped), K_j = kv[key_j, 0:576], V_j = kv[key_j, 0:512] and the upstream
+ * gradient dO = d loss / d out:
+ *   P[h,j]  = exp(scale * q[i,h] . K_j - lse[i,h])
+ *   D[h]    = dO[i,h] . out[i,h]   (its halves over value dims [0,256) and
+ *             [256,512) written to delta[(i*128 + h)*2 + 0] and [... + 1])
+ *   dZ[h,j] = scale * P[h,j] * (dO[i,h] . V_j - D[h])
+ *   d_q[i,h]     = sum_j dZ[h,j] K_j                                  (written)
+ *   d_kv[key_j] += sum_h dZ[h,j] q[i,h];  d_kv[key_j, 0:512] += sum_h P[h,j] dO[i,h]
+ * (d_kv is ACCUMULATED: zero it first for a plain gradient).
+ * in: the forward's attention inputs, BF16, H=128, d_qk=576, d_v=512,
+ * CONTIGUOUS only (DSA_ERR_UNSUPPORTED otherwise). out, lse: the forward's
+ * outputs for this selection; d_out: [n_q, 128, 512] bf16; d_q: [n_q, 128, 576]
+ * bf16; out, d_out, d_q contiguous and 16-byte aligned. d_kv: float32 rows
+ * ld_dkv >= 576 apart (columns 0..575 used); delta: [n_q, 128, 2] float32
+ * scratch, written. The reductions into d_kv make its low-order bits depend
+ * on the order in which queries finish. No workspace. */
+DSA_API dsa_status dsa_sparse_mqa_bwd(const dsa_attn_in* in, const int32_t* idx, int64_t ld_idx,
+                                      int32_t k, const void* out, const float* lse,
+                                      const void* d_out, void* d_q, float* d_kv, int64_t ld_dkv,
+                                      float* delta, dsa_stream_t stream);
+
 /* Workspace bytes for `op` with these inputs (arguments an op does not use may
  * be NULL/0). The workspace must be 256-byte aligned device memory. */
 DSA_API dsa_status dsa_workspace_size(int32_t op, const dsa_indexer_in* indexer,

@@ -15,7 +15,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdsa.so")
 
 SOURCES = ["dsa_api.cu", "indexer_fp8.cu", "topk.cu", "sparse_mqa_bf16.cu", "simt_f32.cu",
-           "indexer_kl.cu"]
+           "indexer_kl.cu", "sparse_mqa_bwd.cu"]
 HEADERS = ["dsa_common.cuh", "dsa_kernels.h", "indexer_epilogue.cuh"]
 
 

@@ -538,6 +538,43 @@ DSA_API dsa_status dsa_indexer_kl(const dsa_attn_in* attn, const int32_t* idx, i
   return DSA_OK;
 }
 
+DSA_API dsa_status dsa_sparse_mqa_bwd(const dsa_attn_in* in, const int32_t* idx, int64_t ld_idx,
+                                      int32_t k, const void* out, const float* lse,
+                                      const void* d_out, void* d_q, float* d_kv, int64_t ld_dkv,
+                                      float* delta, dsa_stream_t stream) {
+  NvtxRange range("dsa_sparse_mqa_bwd");
+  DSA_TRY(check_attn(in));
+  if (in->dtype != DSA_BF16 || in->kv_layout.kind != DSA_KV_CONTIGUOUS) return DSA_ERR_UNSUPPORTED;
+  if (idx == nullptr || out == nullptr || lse == nullptr || d_out == nullptr || d_q == nullptr ||
+      d_kv == nullptr || delta == nullptr || k < 1 || k > kKMax || ld_idx < k || ld_dkv < 576)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(d_out) || !aligned16(d_q)) return DSA_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  DSA_TRY(device_info(&dev));
+  dsa::AttnBwdArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(in->q);
+  a.ld_q = in->ld_q;
+  a.kv = static_cast<const __nv_bfloat16*>(in->kv);
+  a.ld_kv = in->ld_kv;
+  a.idx = idx;
+  a.ld_idx = ld_idx;
+  a.k = k;
+  a.n_q = in->n_q;
+  a.n_keys = in->n_keys;
+  a.scale = in->scale;
+  a.scale_log2 = in->scale * 1.4426950408889634f;
+  a.lse = lse;
+  a.out = static_cast<const __nv_bfloat16*>(out);
+  a.d_out = static_cast<const __nv_bfloat16*>(d_out);
+  a.delta = delta;
+  a.d_q = static_cast<__nv_bfloat16*>(d_q);
+  a.d_kv = d_kv;
+  a.ld_dkv = ld_dkv;
+  a.status = dev->status;
+  DSA_LAUNCH(dsa::launch_attn_bwd(a, reinterpret_cast<cudaStream_t>(stream)));
+  return DSA_OK;
+}
+
 DSA_API dsa_status dsa_workspace_size(int32_t op, const dsa_indexer_in* indexer,
                                       const dsa_attn_in* attn, int32_t n_rows, int32_t n_cols,
                                       int32_t k, size_t* bytes) {
@@ -666,7 +703,7 @@ DSA_API const char* dsa_status_string(dsa_status s) {
 
 DSA_API int32_t dsa_last_cuda_error(void) { return t_last_cuda_error; }
 
-DSA_API int32_t dsa_version(void) { return 200; }
+DSA_API int32_t dsa_version(void) { return 201; }
 
 }  // extern "C"
 

@@ -118,6 +118,31 @@ struct AttnBf16Args {
 
 cudaError_t launch_attn_bf16(const AttnBf16Args& a, cudaStream_t stream);
 
+// Gradient of the sparse MQA attention (contiguous keys; query i at position
+// n_keys - n_q + i): D = rowsum(dO * O), then dq (written) and dkv (accumulated).
+struct AttnBwdArgs {
+  const __nv_bfloat16* q;      // [n_q, 128, 576], query tokens ld_q apart
+  int64_t ld_q;
+  const __nv_bfloat16* kv;     // latent KV rows [n_keys, 576], ld_kv apart
+  int64_t ld_kv;
+  const int32_t* idx;          // [n_q, ld_idx] selected key positions (-1 skipped)
+  int64_t ld_idx;
+  int32_t k;
+  int32_t n_q, n_keys;
+  float scale;                 // softmax scale
+  float scale_log2;            // scale * log2(e)
+  const float* lse;            // [n_q, 128] the forward's natural-log LSE
+  const __nv_bfloat16* out;    // [n_q, 128, 512] the forward's output
+  const __nv_bfloat16* d_out;  // [n_q, 128, 512] upstream gradient
+  float* delta;                // [n_q, 128, 2] written: rowsum(dO * O) over dims [0,256), [256,512)
+  __nv_bfloat16* d_q;          // [n_q, 128, 576] written
+  float* d_kv;                 // [n_keys, ld_dkv] accumulated (columns 0..575)
+  int64_t ld_dkv;
+  int* status;
+};
+
+cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t stream);
+
 struct AttnF32Args {
   const float* q;
   int64_t ld_q;

@@ -34,7 +34,8 @@ DSA_OP_SELECT = 4
 EXPORTED = ["dsa_indexer_scores", "dsa_topk", "dsa_sparse_mqa_fwd", "dsa_select", "dsa_forward",
             "dsa_workspace_size", "dsa_check_status", "dsa_status_string",
             "dsa_last_cuda_error", "dsa_launch_counter", "dsa_version", "dsa_select_noalloc",
-            "dsa_set_wait_limit_ns", "dsa_dense_mqa_fwd", "dsa_select_scored", "dsa_indexer_kl"]
+            "dsa_set_wait_limit_ns", "dsa_dense_mqa_fwd", "dsa_select_scored", "dsa_indexer_kl",
+            "dsa_sparse_mqa_bwd"]
 
 
 class DsaError(RuntimeError):
@@ -83,6 +84,7 @@ def _load():
         "dsa_dense_mqa_fwd": [ctypes.POINTER(AttnIn), P, P, P],
         "dsa_select_scored": [ctypes.POINTER(IndexerIn), I32, P, I64, P, I64, P, SZ, P],
         "dsa_indexer_kl": [ctypes.POINTER(AttnIn), P, I64, I32, P, P, I64, P, P, I64, P],
+        "dsa_sparse_mqa_bwd": [ctypes.POINTER(AttnIn), P, I64, I32, P, P, P, P, P, I64, P, P],
         "dsa_forward": [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), I32, P, P, P, P, SZ, P],
         "dsa_launch_counter": [],
         "dsa_set_wait_limit_ns": [I64],
@@ -235,6 +237,16 @@ def dsa_indexer_kl(attn: _Keep, idx: torch.Tensor, k: int, lse: torch.Tensor,
     _check(LIB.dsa_indexer_kl(ctypes.byref(attn.struct), _ptr(idx), idx.stride(0), k, _ptr(lse),
                               _ptr(sel_scores), sel_scores.stride(0), _ptr(loss), _ptr(grad),
                               grad.stride(0), _stream(stream)), "dsa_indexer_kl")
+
+
+def dsa_sparse_mqa_bwd(attn: _Keep, idx: torch.Tensor, k: int, out: torch.Tensor,
+                       lse: torch.Tensor, d_out: torch.Tensor, d_q: torch.Tensor,
+                       d_kv: torch.Tensor, delta: torch.Tensor, stream=None):
+    """Gradient of dsa_sparse_mqa_fwd: writes d_q and delta, ADDS into d_kv."""
+    _check(LIB.dsa_sparse_mqa_bwd(ctypes.byref(attn.struct), _ptr(idx), idx.stride(0), k,
+                                  _ptr(out), _ptr(lse), _ptr(d_out), _ptr(d_q), _ptr(d_kv),
+                                  d_kv.stride(0), _ptr(delta), _stream(stream)),
+           "dsa_sparse_mqa_bwd")
 
 
 def dsa_select(ind: _Keep, k: int, idx: torch.Tensor, ws: torch.Tensor, stream=None):

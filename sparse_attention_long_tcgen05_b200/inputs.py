@@ -191,6 +191,39 @@ def make_decode(wl: Workload, device="cpu", seed: int = 0, ctx_lens=None) -> Dec
         kv_cache.view(num_pages, PAGE, wl.D_K))
 
 
+def make_grad_out(n_q: int, H: int = 128, d_v: int = 512, device="cpu", seed: int = 0):
+    """Seeded upstream gradient dO [n_q, H, d_v] for the attention backward:
+    bf16 draws of N(0, 1), row-chunked like the other bf16 tensors."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return _randn((n_q, H, d_v), gen, device, dtype=torch.bfloat16, chunk_rows=2048)
+
+
+def random_selection(n_q: int, n_keys: int, k: int, device="cpu", seed: int = 0,
+                     chunk_rows: int = 8192) -> torch.Tensor:
+    """Seeded valid selection in the top-k's output format, for testing the
+    attention alone: query i (position p = n_keys - n_q + i) keeps every key
+    0..p when p < k, else one key drawn uniformly from each of k consecutive
+    strata [floor(j w), floor((j+1) w)) of 0..p, w = (p+1)/k -- k distinct keys,
+    ascending, spread over the whole prefix. Padded with -1 to k columns."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    idx = torch.empty(n_q, k, dtype=torch.int32, device=device)
+    j = torch.arange(k, device=device, dtype=torch.float64)
+    for r0 in range(0, n_q, chunk_rows):
+        r1 = min(n_q, r0 + chunk_rows)
+        pos = torch.arange(n_keys - n_q + r0, n_keys - n_q + r1, device=device,
+                           dtype=torch.float64)[:, None]
+        w = (pos + 1.0) / k
+        lo = torch.floor(j * w)
+        hi = torch.floor((j + 1.0) * w)
+        u = torch.rand((r1 - r0, k), generator=gen, device=device, dtype=torch.float64)
+        sparse = lo + torch.floor(u * (hi - lo))
+        dense = torch.where(j <= pos, j, torch.full_like(j, -1.0))
+        idx[r0:r1] = torch.where(pos + 1.0 > k, sparse, dense).to(torch.int32)
+    return idx
+
+
 def sample_rows(L: int, n: int = 512, seed: int = 1, k: int = 2048):
     """Seeded row sample for large prefill checks: {0, k-1, k, L-1} plus
     uniform draws, sorted and unique."""

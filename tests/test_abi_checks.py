@@ -303,6 +303,27 @@ def test_kl_and_select_scored_checks(dsa):
     _expect(dsa, UNS, lambda: dense(attn=_mut(f32, n_keys=5000, n_q=100)))   # fp32 dense > 4096 keys
 
 
+def test_backward_checks(dsa):
+    att = _attn(dsa)
+    INV, UNS = dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_UNSUPPORTED
+    P = FAKE + 0x200000
+
+    def bwd(attn=att, idx=P, ld_idx=2048, k=2048, out=P + 0x1000, lse=P, d_out=P + 0x2000,
+            d_q=P + 0x3000, d_kv=P, ld_dkv=576, delta=P):
+        return dsa.LIB.dsa_sparse_mqa_bwd(ctypes.byref(attn), _p(idx), ld_idx, k, _p(out),
+                                          _p(lse), _p(d_out), _p(d_q), _p(d_kv), ld_dkv,
+                                          _p(delta), None)
+    _expect(dsa, dsa.DSA_ERR_CUDA, lambda: bwd())
+    for kw in (dict(idx=None), dict(out=None), dict(lse=None), dict(d_out=None), dict(d_q=None),
+               dict(d_kv=None), dict(delta=None), dict(k=0), dict(k=2049), dict(ld_idx=100),
+               dict(ld_dkv=575), dict(out=P + 0x1008), dict(d_out=P + 0x2008),
+               dict(d_q=P + 0x3004)):
+        _expect(dsa, INV, lambda: bwd(**kw))
+    f32 = _mut(att, dtype=dsa.DSA_F32, heads=8, d_qk=64, d_v=64, ld_q=512, ld_kv=64)
+    _expect(dsa, UNS, lambda: bwd(attn=f32))
+    _expect(dsa, UNS, lambda: bwd(attn=_attn(dsa, kv=_paged(dsa), n_q=64)))
+
+
 def test_nvtx_ranges_switch_on_without_a_profiler():
     """DSA_NVTX=1 turns the per-call and per-block NVTX ranges on (read once
     per process); with no profiler attached they are no-ops and the call
