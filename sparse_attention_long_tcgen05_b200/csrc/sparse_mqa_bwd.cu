@@ -40,9 +40,11 @@
 //      MN-major straight from the tiles above), and the 64 rope dims (M padded
 //      to 128; the extra rows are never read), into the TMEM columns of S and dP
 //      (free by then) and 64 spare ones;
-//   5. four drain warps read those tiles (TMEM lane = dim, column = key) and add
-//      them into dkv with fp32 reductions, 32 consecutive dims of one row per
-//      warp instruction; a CTA adds the rope dims of its own 32 keys only.
+//   5. eight warps (the four drain warps and the four P / dZ warps, which are
+//      idle until the next block's S) read those tiles (TMEM lane = dim,
+//      column = key), release the S and dP columns before any reduction, and
+//      add them into dkv with fp32 reductions, 32 consecutive dims of one row
+//      per warp instruction; a CTA adds the rope dims of its own 32 keys only.
 // TMEM (512 columns): dq [0,256), rope dq partial [256,320), S [320,384),
 // dP [384,448), rope dkv tile [448,512).
 //
@@ -50,8 +52,10 @@
 //   warps 0-7    plan (four 64-entry blocks of the index row each), then with
 //                warps 9-11 the cp.async gather;
 //   warp 8       owns TMEM and issues the MMAs;
-//   warps 12-15  exchange and P / dZ (thread = head = TMEM lane);
-//   warps 16-19  dkv drain, then the dq epilogue (thread = TMEM lane).
+//   warps 12-15  exchange and P / dZ (thread = head = TMEM lane), then key
+//                columns 0-31 of the block's dkv drain;
+//   warps 16-19  key columns 32-63 of the dkv drain, then the dq epilogue
+//                (thread = TMEM lane).
 #include <cuda_fp16.h>
 
 #include "dsa_common.cuh"
@@ -124,6 +128,59 @@ __device__ __forceinline__ uint32_t sw_off(int r, int u) {
   return static_cast<uint32_t>(r * 128 + ((u ^ (r & 7)) << 4));
 }
 
+// One of the eight workers draining block j's dkv^T tiles: TMEM sub-partition
+// s (lanes = dims 32s ..), key columns 32 half .. 32 half + 31. Each value tile
+// is released as soon as all workers have read it (the S columns first, whose
+// MMA for the next block runs while the dP columns are drained), the fp32
+// reductions follow (the key's KV row broadcast from the lane that read it);
+// then the rope tile (lanes 0-63; this CTA's 32 keys, 16 per worker).
+__device__ __forceinline__ bool drain_block(Smem& S, const AttnBwdArgs& a, uint32_t tmem_base,
+                                            int s, int half, int lane, int j, uint32_t rank,
+                                            int col0) {
+  if (!mbar_wait_warp(&S.dkv_full, static_cast<uint32_t>(j) & 1u, a.status)) return false;
+  tc_fence_after();
+  const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(32 * s) << 16);
+  const int* rb = S.rows + S.blk[j] * kBK;
+  const int64_t ld = a.ld_dkv;
+  const int dl = 32 * s + lane;
+  const int my_row = rb[32 * half + lane];
+  const uint32_t mk = S.mask[j][half];
+#pragma unroll 1
+  for (int t = 0; t < 2; ++t) {
+    uint32_t v[32];
+    tmem_ld32(t_lane + (t ? kColDP : kColS) + 32 * half, v);
+    tmem_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(t ? &S.dp_free : &S.s_free);
+    float* const d = a.d_kv + col0 + 128 * t + dl;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int64_t row = __shfl_sync(0xffffffffu, my_row, i);
+      if ((mk >> i) & 1u) atomicAdd(d + row * ld, __uint_as_float(v[i]));
+    }
+  }
+  uint32_t x[16];
+  if (s < 2) {
+    tmem_ld16(t_lane + kColX + 32u * rank + 16 * half, x);
+    tmem_wait_ld();
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&S.x_free);
+  if (s < 2) {
+    const int r_row = rb[32 * static_cast<int>(rank) + 16 * half + (lane & 15)];
+    const uint32_t mr = (S.mask[j][rank] >> (16 * half)) & 0xffffu;
+    float* const dr = a.d_kv + 512 + dl;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int64_t row = __shfl_sync(0xffffffffu, r_row, i);
+      if ((mr >> i) & 1u) atomicAdd(dr + row * ld, __uint_as_float(x[i]));
+    }
+  }
+  return true;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -159,9 +216,9 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
     mbar_init(&S.pdz_full, 4);
     mbar_init(&S.peer_free, 1);     // the peer's MMA commit
     mbar_init(&S.dkv_full, 1);
-    mbar_init(&S.s_free, 4);
-    mbar_init(&S.dp_free, 4);
-    mbar_init(&S.x_free, 4);
+    mbar_init(&S.s_free, 8);
+    mbar_init(&S.dp_free, 8);
+    mbar_init(&S.x_free, 8);
     mbar_init(&S.dq_full, 1);
     mbar_init(&S.rq_full, 1);
     fence_barrier_init();
@@ -283,9 +340,8 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
       const uint32_t ph = static_cast<uint32_t>(j) & 1u;
       const uint32_t pp = ph ^ 1u;
       ok = mbar_wait_warp(&S.kv_full, ph, a.status);
-      // the drain has read block j-1's dkv tiles out of the S and dP columns
-      if (ok && j > 0)
-        ok = mbar_wait_warp(&S.s_free, pp, a.status) && mbar_wait_warp(&S.dp_free, pp, a.status);
+      // the drain has read block j-1's first dkv tile out of the S columns
+      if (ok && j > 0) ok = mbar_wait_warp(&S.s_free, pp, a.status);
       if (!ok) break;
       tc_fence_after();
       if (lane == 0) {
@@ -301,6 +357,15 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tS + 32u * rank, qr + 2 * kk, rd + 2 * kk, id_sr, 1u);
+      }
+      __syncwarp();
+      // ... and the second out of the dP columns
+      if (j > 0 && !mbar_wait_warp(&S.dp_free, pp, a.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (lane == 0) {
         for (int c = 0; c < 4; ++c) {
           const uint64_t od = sw128_desc(smem_u32(S.dout[c]), 16, 1024);
           const uint64_t kd = sw128_desc(smem_u32(S.kv[c]), 16, 1024);
@@ -454,6 +519,11 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.pdz_full);
+      // idle until the next block's S: drain half of this block's dkv tiles
+      if (!drain_block(S, a, tmem_base, s, 0, lane, j, rank, col0)) {
+        ok = false;
+        break;
+      }
     }
   } else {
     // ------------------------------------------------------------ dkv drain, dq epilogue
@@ -462,54 +532,8 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(32 * s) << 16);
     bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
     const int n = ok ? S.n_blocks : 0;
-    const int64_t ld = a.ld_dkv;
-    for (int j = 0; j < n && ok; ++j) {
-      if (!mbar_wait_warp(&S.dkv_full, static_cast<uint32_t>(j) & 1u, a.status)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const int* rb = S.rows + S.blk[j] * kBK;
-      const uint32_t mk0 = S.mask[j][0];
-      const uint32_t mk1 = S.mask[j][1];
-#pragma unroll 1
-      for (int t = 0; t < 2; ++t) {
-        uint32_t v0[32], v1[32];
-        const uint32_t col = t ? kColDP : kColS;
-        tmem_ld32(t_lane + col, v0);
-        tmem_ld32(t_lane + col + 32, v1);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(t ? &S.dp_free : &S.s_free);
-        float* const dst = a.d_kv + col0 + 128 * t + dl;
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if ((mk0 >> i) & 1u) atomicAdd(dst + rb[i] * ld, __uint_as_float(v0[i]));
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if ((mk1 >> i) & 1u) atomicAdd(dst + rb[32 + i] * ld, __uint_as_float(v1[i]));
-      }
-      {
-        // rope dims (lanes 0-63) of this CTA's 32 keys
-        uint32_t v[32];
-        if (s < 2) {
-          tmem_ld32(t_lane + kColX + 32u * rank, v);
-          tmem_wait_ld();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.x_free);
-        if (s < 2) {
-          const uint32_t mk = rank ? mk1 : mk0;
-          const int* rr = rb + 32 * static_cast<int>(rank);
-          float* const dst = a.d_kv + 512 + dl;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if ((mk >> i) & 1u) atomicAdd(dst + rr[i] * ld, __uint_as_float(v[i]));
-        }
-      }
-    }
+    for (int j = 0; j < n && ok; ++j)
+      ok = drain_block(S, a, tmem_base, s, 1, lane, j, rank, col0);
     // dq of head dl: value dims col0 .. col0+255 here; the rope dims of the
     // CTA's own 64 heads (64 rank ..) with the peer's partial added
     const bool got = mbar_wait_warp(&S.dq_full, 0, a.status);
