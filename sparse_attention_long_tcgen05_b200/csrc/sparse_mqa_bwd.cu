@@ -40,22 +40,25 @@
 //      MN-major straight from the tiles above), and the 64 rope dims (M padded
 //      to 128; the extra rows are never read), into the TMEM columns of S and dP
 //      (free by then) and 64 spare ones;
-//   5. eight warps (the four drain warps and the four P / dZ warps, which are
-//      idle until the next block's S) read those tiles (TMEM lane = dim,
-//      column = key), release the S and dP columns before any reduction, and
-//      add them into dkv with fp32 reductions, 32 consecutive dims of one row
-//      per warp instruction; a CTA adds the rope dims of its own 32 keys only.
+//   5. eight of the gather warps, idle from the moment the next block's rows
+//      have landed, read those tiles (TMEM lane = dim, column = key), release
+//      the S and dP columns to the next block's MMAs as soon as each is read,
+//      and add them into dkv with fp32 reductions, 32 consecutive dims of one
+//      row per warp instruction; a CTA adds the rope dims of its own 32 keys
+//      only. The reductions (576 fp32 adds per selected pair) thus stay off the
+//      chain MMA -> exchange -> P / dZ -> MMA that sets the pace.
 // TMEM (512 columns): dq [0,256), rope dq partial [256,320), S [320,384),
 // dP [384,448), rope dkv tile [448,512).
 //
 // Roles (20 warps):
 //   warps 0-7    plan (four 64-entry blocks of the index row each), then with
-//                warps 9-11 the cp.async gather;
+//                warps 9-11 the cp.async gather; after gathering block j they
+//                drain block j-1's dkv tiles (warps w and w+4: TMEM
+//                sub-partition w, key columns 0-31 and 32-63);
 //   warp 8       owns TMEM and issues the MMAs;
-//   warps 12-15  exchange and P / dZ (thread = head = TMEM lane), then key
-//                columns 0-31 of the block's dkv drain;
-//   warps 16-19  key columns 32-63 of the dkv drain, then the dq epilogue
-//                (thread = TMEM lane).
+//   warps 12-19  exchange and P / dZ (thread = head = TMEM lane; warps 12-15
+//                keys 0-31 of each block, 16-19 keys 32-63); warps 16-19 then
+//                write dq.
 #include <cuda_fp16.h>
 
 #include "dsa_common.cuh"
@@ -74,8 +77,7 @@ constexpr int kChunkKV = kBK * 128;   // 64 dims of a block's 64 rows: 8 KB
 constexpr int kPlanWarps = 8;
 constexpr int kMmaWarp = 8;
 constexpr int kGatherWarps = 11;      // warps 0-7 and 9-11
-constexpr int kSoftWarp0 = 12;        // 12..15
-constexpr int kDrainWarp0 = 16;       // 16..19
+constexpr int kSoftWarp0 = 12;        // 12..19: exchange, P and dZ
 constexpr int kThreads = 20 * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDQ = 0;
@@ -100,7 +102,7 @@ struct __align__(1024) Smem {
   uint32_t mask[kMaxBlocks][2];   // valid entries of the j-th non-empty block
   int32_t blk[kMaxBlocks];        // block number of the j-th non-empty block
   int32_t n_blocks;
-  uint64_t plan_full, q_full, kv_full, kv_empty, sdp_full, rx_full, pdz_full;
+  uint64_t plan_full, q_full, kv_full, kv_empty, s_full, sdp_full, rx_full, pdz_full;
   uint64_t peer_free;   // the peer's MMAs of a block are done: its P / dZ tiles may be written
   uint64_t dkv_full, s_free, dp_free, x_free, dq_full, rq_full;
   uint32_t tmem_base;
@@ -211,9 +213,10 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
     mbar_init(&S.q_full, kGatherWarps);
     mbar_init(&S.kv_full, kGatherWarps);
     mbar_init(&S.kv_empty, 1);
+    mbar_init(&S.s_full, 1);
     mbar_init(&S.sdp_full, 1);
     mbar_init(&S.rx_full, 1);       // one expect-tx arrival; the peer's st.async bytes
-    mbar_init(&S.pdz_full, 4);
+    mbar_init(&S.pdz_full, 8);
     mbar_init(&S.peer_free, 1);     // the peer's MMA commit
     mbar_init(&S.dkv_full, 1);
     mbar_init(&S.s_free, 8);
@@ -296,6 +299,11 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
     const int n = ok0 ? S.n_blocks : 0;
     const char* kvb = reinterpret_cast<const char*>(a.kv);
     const int64_t ldb = a.ld_kv * 2;
+    // warps 0-7 also drain: block j-1's dkv tiles land about when the copies
+    // of block j have been issued and have landed
+    const bool drains = warp < kPlanWarps;
+    bool dok = true;
+    int gathered = 0;
     for (int j = 0; j < n; ++j) {
       if (j > 0 && !mbar_wait_warp(&S.kv_empty, static_cast<uint32_t>(j - 1) & 1u, a.status))
         break;
@@ -320,8 +328,12 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.kv_full);
+      gathered = j + 1;
+      if (drains && j > 0 && dok) dok = drain_block(S, a, tmem_base, warp & 3, warp >> 2, lane, j - 1, rank, col0);
     }
     cp_async_wait_group<0>();
+    if (drains && dok && n > 0 && gathered == n)
+      drain_block(S, a, tmem_base, warp & 3, warp >> 2, lane, n - 1, rank, col0);
   } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------- MMA issuer
     const uint32_t id_s = make_idesc(kBK, 1, 1, 0, 0);        // K-major A and B
@@ -357,6 +369,7 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tS + 32u * rank, qr + 2 * kk, rd + 2 * kk, id_sr, 1u);
+        mma_commit(&S.s_full);   // the partial S travels while dP is computed
       }
       __syncwarp();
       // ... and the second out of the dP columns
@@ -418,10 +431,13 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
     }
     if (lane == 0) mma_commit(&S.dq_full);
     __syncwarp();
-  } else if (warp < kDrainWarp0) {
+  } else {
     // ------------------------------------------------------------ exchange, P and dZ
-    const int s = warp - kSoftWarp0;          // TMEM sub-partition
+    // warps 12-15 take keys 0-31 of every block, warps 16-19 keys 32-63
+    const int s = warp & 3;                   // TMEM sub-partition
+    const int kh = (warp - kSoftWarp0) >> 2;  // key half
     const int m = 32 * s + lane;              // head = TMEM lane = tile row
+    const int dl = m;
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(32 * s) << 16);
     const int sw = m & 7;
     const uint32_t row_off = static_cast<uint32_t>((m >> 3) * 1024 + (m & 7) * 128);
@@ -441,8 +457,8 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
     const int n = ok ? S.n_blocks : 0;
     for (int j = 0; j < n && ok; ++j) {
       const uint32_t ph = static_cast<uint32_t>(j) & 1u;
-      if (s == 0 && lane == 0) mbar_arrive_expect_tx(&S.rx_full, kRxBytes);
-      if (!mbar_wait_warp(&S.sdp_full, ph, a.status)) {
+      if (warp == kSoftWarp0 && lane == 0) mbar_arrive_expect_tx(&S.rx_full, kRxBytes);
+      if (!mbar_wait_warp(&S.s_full, ph, a.status)) {
         ok = false;
         break;
       }
@@ -453,10 +469,10 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
       }
       tc_fence_after();
 #pragma unroll 1
-      for (int hf = 0; hf < 4; ++hf) {   // 16 keys at a time
-        uint32_t v[16], u[16];
+      for (int hh = 0; hh < 2; ++hh) {   // partial S, 16 keys at a time
+        const int hf = 2 * kh + hh;
+        uint32_t v[16];
         tmem_ld16(t_lane + kColS + 16 * hf, v);
-        tmem_ld16(t_lane + kColDP + 16 * hf, u);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -466,6 +482,22 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
                                  pack_half2(v[8 * c + 4], v[8 * c + 5]),
                                  pack_half2(v[8 * c + 6], v[8 * c + 7])),
                       rx_full_peer);
+        }
+      }
+      if (!mbar_wait_warp(&S.sdp_full, ph, a.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {   // partial dP - D
+        const int hf = 2 * kh + hh;
+        uint32_t u[16];
+        tmem_ld16(t_lane + kColDP + 16 * hf, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t off = static_cast<uint32_t>(((2 * hf + c) ^ sw) << 4);
           uint32_t du[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) du[e] = __float_as_uint(__uint_as_float(u[8 * c + e]) - dlt);
@@ -479,15 +511,15 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
         ok = false;
         break;
       }
-      const uint32_t mk0 = S.mask[j][0];
-      const uint32_t mk1 = S.mask[j][1];
+      const uint32_t mkh = S.mask[j][kh];
 #pragma unroll 1
-      for (int hf = 0; hf < 4; ++hf) {
+      for (int hh = 0; hh < 2; ++hh) {
+        const int hf = 2 * kh + hh;
         uint32_t v[16], u[16];
         tmem_ld16(t_lane + kColS + 16 * hf, v);
         tmem_ld16(t_lane + kColDP + 16 * hf, u);
         tmem_wait_ld();
-        const uint32_t mk = ((hf < 2 ? mk0 : mk1) >> (16 * (hf & 1))) & 0xffffu;
+        const uint32_t mk = (mkh >> (16 * hh)) & 0xffffu;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const uint32_t off = static_cast<uint32_t>(((2 * hf + c) ^ sw) << 4);
@@ -519,83 +551,71 @@ sparse_mqa_bwd_kernel(const __grid_constant__ AttnBwdArgs a) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.pdz_full);
-      // idle until the next block's S: drain half of this block's dkv tiles
-      if (!drain_block(S, a, tmem_base, s, 0, lane, j, rank, col0)) {
-        ok = false;
-        break;
-      }
     }
-  } else {
-    // ------------------------------------------------------------ dkv drain, dq epilogue
-    const int s = warp - kDrainWarp0;
-    const int dl = 32 * s + lane;             // TMEM lane
-    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(32 * s) << 16);
-    bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
-    const int n = ok ? S.n_blocks : 0;
-    for (int j = 0; j < n && ok; ++j)
-      ok = drain_block(S, a, tmem_base, s, 1, lane, j, rank, col0);
-    // dq of head dl: value dims col0 .. col0+255 here; the rope dims of the
-    // CTA's own 64 heads (64 rank ..) with the peer's partial added
-    const bool got = mbar_wait_warp(&S.dq_full, 0, a.status);
-    const bool live = ok && got && n > 0;
-    if (got) tc_fence_after();
-    __nv_bfloat16* const dqrow = a.d_q + (static_cast<int64_t>(qi) * kH + dl) * 576;
+    if (kh == 1) {
+      // dq of head dl: value dims col0 .. col0+255 here; the rope dims of the
+      // CTA's own 64 heads (64 rank ..) with the peer's partial added
+      const bool got = mbar_wait_warp(&S.dq_full, 0, a.status);
+      const bool live = ok && got && n > 0;
+      if (got) tc_fence_after();
+      __nv_bfloat16* const dqrow = a.d_q + (static_cast<int64_t>(qi) * kH + dl) * 576;
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-      uint32_t v[32];
-      if (live) {
-        tmem_ld32(t_lane + kColDQ + 32 * c, v);
-        tmem_wait_ld();
-      }
-      uint4* dst = reinterpret_cast<uint4*>(dqrow + col0 + 32 * c);
+      for (int c = 0; c < 8; ++c) {
+        uint32_t v[32];
+        if (live) {
+          tmem_ld32(t_lane + kColDQ + 32 * c, v);
+          tmem_wait_ld();
+        }
+        uint4* dst = reinterpret_cast<uint4*>(dqrow + col0 + 32 * c);
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        dst[i] = live ? make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
-                                   pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
-                                   pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
-                                   pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])))
-                      : make_uint4(0u, 0u, 0u, 0u);
-    }
-    const bool own = (s >> 1) == static_cast<int>(rank);   // heads 64 rank .. 64 rank + 63
-    // slot of head dl in its owner's exchange area (the owner's P tile)
-    const uint32_t slot_off = static_cast<uint32_t>((dl & 63) * 256);
-    if (!own) {
-      // the peer's last MMAs are done: its P tile takes our partials
-      if (live && mbar_wait_cluster_warp(&S.peer_free, static_cast<uint32_t>(n - 1) & 1u, a.status)) {
-        const uint32_t dst = mapa_shared(smem_u32(S.p) + slot_off, peer);
-        const uint32_t bar = mapa_shared(smem_u32(&S.rq_full), peer);
+        for (int i = 0; i < 4; ++i)
+          dst[i] = live ? make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
+                                     pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                                     pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                                     pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])))
+                        : make_uint4(0u, 0u, 0u, 0u);
+      }
+      const bool own = (s >> 1) == static_cast<int>(rank);   // heads 64 rank .. 64 rank + 63
+      // slot of head dl in its owner's exchange area (the owner's P tile)
+      const uint32_t slot_off = static_cast<uint32_t>((dl & 63) * 256);
+      if (!own) {
+        // the peer's last MMAs are done: its P tile takes our partials
+        if (live && mbar_wait_cluster_warp(&S.peer_free, static_cast<uint32_t>(n - 1) & 1u, a.status)) {
+          const uint32_t dst = mapa_shared(smem_u32(S.p) + slot_off, peer);
+          const uint32_t bar = mapa_shared(smem_u32(&S.rq_full), peer);
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[32];
+            tmem_ld32(t_lane + kColDQR + 32 * h, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              st_async_v4(dst + 128 * h + 16 * i,
+                          make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]), bar);
+          }
+        }
+      } else {
+        if (live && s == 2 * static_cast<int>(rank) && lane == 0)
+          mbar_arrive_expect_tx(&S.rq_full, kRqBytes);
+        const bool x_ok = live && mbar_wait_cluster_warp(&S.rq_full, 0, a.status);
+        const float* px = reinterpret_cast<const float*>(S.p + slot_off);
+        uint4* dst = reinterpret_cast<uint4*>(dqrow + 512);
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           uint32_t r[32];
-          tmem_ld32(t_lane + kColDQR + 32 * h, r);
-          tmem_wait_ld();
+          if (x_ok) {
+            tmem_ld32(t_lane + kColDQR + 32 * h, r);
+            tmem_wait_ld();
+          }
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            st_async_v4(dst + 128 * h + 16 * i,
-                        make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]), bar);
-        }
-      }
-    } else {
-      if (live && s == 2 * static_cast<int>(rank) && lane == 0)
-        mbar_arrive_expect_tx(&S.rq_full, kRqBytes);
-      const bool x_ok = live && mbar_wait_cluster_warp(&S.rq_full, 0, a.status);
-      const float* px = reinterpret_cast<const float*>(S.p + slot_off);
-      uint4* dst = reinterpret_cast<uint4*>(dqrow + 512);
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        uint32_t r[32];
-        if (x_ok) {
-          tmem_ld32(t_lane + kColDQR + 32 * h, r);
-          tmem_wait_ld();
-        }
+          for (int i = 0; i < 4; ++i) {
+            float f[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float f[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            f[e] = x_ok ? __uint_as_float(r[8 * i + e]) + px[32 * h + 8 * i + e] : 0.f;
-          dst[4 * h + i] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                      pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+            for (int e = 0; e < 8; ++e)
+              f[e] = x_ok ? __uint_as_float(r[8 * i + e]) + px[32 * h + 8 * i + e] : 0.f;
+            dst[4 * h + i] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                        pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+          }
         }
       }
     }
