@@ -513,6 +513,38 @@ def attention_backward(dsa, wl, att, idx, out, lse, k, world, peaks, steps=2):
                    "the 128K selection of dsa_forward; dkv accumulated in fp32"}
 
 
+def profile_backward(L: int):
+    """The attention backward alone on an L-token prefill of the 128K
+    workload's shapes (seeded inputs; selection from random_selection), one
+    warm-up launch and three timed ones: the command the backward's ncu
+    summaries are taken with."""
+    import dataclasses
+    from sparse_attention_long_tcgen05_b200 import dsa
+    from sparse_attention_long_tcgen05_b200.inputs import (WORKLOADS, make_grad_out,
+                                                           make_prefill, random_selection)
+    wl = dataclasses.replace(WORKLOADS[3], name=f"prefill_L{L}", L=L)
+    k = wl.k
+    inp = make_prefill(wl, device="cuda", seed=0)
+    idx = random_selection(L, L, k, device="cuda", seed=70)
+    d_out = make_grad_out(L, wl.H, wl.D_V, device="cuda", seed=71)
+    att = dsa.attn_in(inp.q, inp.kv, wl.scale, wl.D_V)
+    out = torch.empty(L, wl.H, wl.D_V, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(L, wl.H, device="cuda")
+    dsa.dsa_sparse_mqa_fwd(att, idx, k, out, lse)
+    dq = torch.empty(L, wl.H, wl.D_K, dtype=torch.bfloat16, device="cuda")
+    dkv = torch.zeros(L, wl.D_K, device="cuda")
+    delta = torch.empty(L, wl.H, 2, device="cuda")
+    run = lambda: dsa.dsa_sparse_mqa_bwd(att, idx, k, out, lse, d_out, dq, dkv, delta)
+    ms = timed(run, 3, 1, 1)
+    st = dsa.dsa_check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {dsa.status_string(st)}")
+    pairs = int((idx >= 0).sum())
+    tf = 2.0 * wl.H * (2 * wl.D_K + wl.D_K + 2 * wl.D_V) * pairs / (ms * 1e-3) / 1e12
+    return {"profile": "attention_backward", "L": L, "k": k, "ms": ms, "pairs": pairs,
+            "bf16_tflops": tf}
+
+
 def prefill_e2e(dsa, inp, ind, att, ws, idx, out, lse, k, args, world, n_chunks=8):
     """Same metric through the public calls with HOST buffers: every step copies
     all of its inputs from pinned host memory and reads the attention output and
@@ -752,6 +784,10 @@ def main():
     ap.add_argument("--skip-fp8-peak", action="store_true",
                     help="do not measure the FP8 GEMM peak (the indexer is then reported "
                          "against 2 x the bf16 peak)")
+    ap.add_argument("--profile-bwd", type=int, default=0, metavar="L",
+                    help="run only the attention backward on an L-token prefill (seeded "
+                         "inputs, random_selection), warm-up then 3 timed launches: a "
+                         "profiling aid with no headline value")
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=10.0)
@@ -764,6 +800,9 @@ def main():
         if rank != 0:
             return
         print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return
+    if args.profile_bwd:
+        print(json.dumps(profile_backward(args.profile_bwd)), flush=True)
         return
     world, rank, local = dist_setup()
     res = run_ours(args, world, rank, local)

@@ -131,11 +131,12 @@ __device__ __forceinline__ uint32_t sw_off(int r, int u) {
 }
 
 // One of the eight workers draining block j's dkv^T tiles: TMEM sub-partition
-// s (lanes = dims 32s ..), key columns 32 half .. 32 half + 31. Each value tile
-// is released as soon as all workers have read it (the S columns first, whose
-// MMA for the next block runs while the dP columns are drained), the fp32
-// reductions follow (the key's KV row broadcast from the lane that read it);
-// then the rope tile (lanes 0-63; this CTA's 32 keys, 16 per worker).
+// s (lanes = dims 32s ..), key columns 32 half .. 32 half + 31. Both value
+// tiles are read before anything else, so that the next block's S and dP MMAs
+// can take their columns at once; the fp32 reductions follow (the key's KV row
+// broadcast from the lane that read it); then the rope tile (lanes 0-63; this
+// CTA's 32 keys, 16 per worker), whose columns are needed only by the next
+// block's dkv MMAs.
 __device__ __forceinline__ bool drain_block(Smem& S, const AttnBwdArgs& a, uint32_t tmem_base,
                                             int s, int half, int lane, int j, uint32_t rank,
                                             int col0) {
@@ -145,21 +146,28 @@ __device__ __forceinline__ bool drain_block(Smem& S, const AttnBwdArgs& a, uint3
   const int* rb = S.rows + S.blk[j] * kBK;
   const int64_t ld = a.ld_dkv;
   const int dl = 32 * s + lane;
-  const int my_row = rb[32 * half + lane];
-  const uint32_t mk = S.mask[j][half];
-#pragma unroll 1
-  for (int t = 0; t < 2; ++t) {
-    uint32_t v[32];
-    tmem_ld32(t_lane + (t ? kColDP : kColS) + 32 * half, v);
+  {
+    uint32_t v0[32], v1[32];
+    tmem_ld32(t_lane + kColS + 32 * half, v0);
+    tmem_ld32(t_lane + kColDP + 32 * half, v1);
     tmem_wait_ld();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(t ? &S.dp_free : &S.s_free);
-    float* const d = a.d_kv + col0 + 128 * t + dl;
+    if (lane == 0) {
+      mbar_arrive(&S.s_free);
+      mbar_arrive(&S.dp_free);
+    }
+    const int my_row = rb[32 * half + lane];
+    const uint32_t mk = S.mask[j][half];
+    float* const d0 = a.d_kv + col0 + dl;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int64_t row = __shfl_sync(0xffffffffu, my_row, i);
-      if ((mk >> i) & 1u) atomicAdd(d + row * ld, __uint_as_float(v[i]));
+      if ((mk >> i) & 1u) {
+        float* const p = d0 + row * ld;
+        atomicAdd(p, __uint_as_float(v0[i]));
+        atomicAdd(p + 128, __uint_as_float(v1[i]));
+      }
     }
   }
   uint32_t x[16];
