@@ -73,7 +73,7 @@ namespace {
 constexpr int kH = 128;              // query heads = MMA M
 constexpr int kBK = 64;              // keys per block = QK^T MMA N
 constexpr int kStages = 4;           // ring of the four 64-dim value chunks of a key block
-constexpr int kRopeStages = 2;       // ring of the rope chunk of this CTA's 32 keys
+constexpr int kRopeStages = 4;       // ring of the rope chunk of this CTA's 32 keys
 constexpr int kChunkKV = kBK * 128;  // one 64-dim chunk of a key block: 64 rows x 128 B
 constexpr int kMaxK = 2048;
 constexpr int kMaxBlocks = kMaxK / kBK;
@@ -104,7 +104,7 @@ constexpr uint32_t kRxPBytes = 64 * 128 + 64 * 4;   // the peer's 64 P rows + re
 
 struct __align__(1024) Smem {
   uint8_t kv[kStages][4][kChunkKV];           // 128 KB value-chunk ring
-  uint8_t rope[kRopeStages][kChunkKV / 2];    // 8 KB: rope dims of this CTA's 32 keys
+  uint8_t rope[kRopeStages][kChunkKV / 2];    // 16 KB: rope dims of this CTA's 32 keys
   uint8_t p[2][kH * 128];                     // 2 x 16 KB: P [128 rows x 64 keys] bf16
   uint32_t rx_s[64 * kBK / 2];                // 8 KB: the peer's partial S of our heads (fp16 pairs)
   uint32_t tx_s[64 * kBK / 2];                // 8 KB: our partial S of the peer's heads (fp16 pairs)
