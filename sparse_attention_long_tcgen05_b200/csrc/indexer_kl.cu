@@ -20,14 +20,18 @@
 //   warps 0-7    plan (index row -> physical rows, valid masks, non-empty
 //                blocks), then copy each block's 64 selected rows (1152 B each)
 //                with 16-byte cp.async into nine 128-byte-swizzled 64-dim
-//                tiles, two stages;
+//                tiles, three stages (216 KB: the copies are latency-bound,
+//                and with two stages the copy of block j could start only
+//                once S of block j-2 was done -- 95.7 -> 72.6 ms at 128K);
 //   warp 8       owns TMEM and issues S = Q K^T (M = 128 heads, N = 64 keys,
 //                K = 576 in 36 steps of 16) into the S buffer of the block;
 //   warps 12-15  stage Q in TMEM (thread = head), then per block read S, form
 //                exp(scale s - lse) for their 32 heads and sum them over the
 //                heads (a shuffle transpose-reduce within the warp, then the
-//                four warps' partial sums in shared memory) into p; at the end
-//                the indexer's softmax, the loss and the gradient.
+//                four warps' partial sums in shared memory) into p, which
+//                waits in the gradient row (L2-resident global memory, leaving
+//                the shared memory to the copies); at the end the indexer's
+//                softmax, the loss and the gradient, written over p.
 #include "dsa_common.cuh"
 #include "dsa_kernels.h"
 
@@ -40,7 +44,7 @@ constexpr int kMaxK = 2048;
 constexpr int kMaxBlocks = kMaxK / kBK;
 constexpr int kChunks = 9;                      // 64-dim chunks of a 576-wide row
 constexpr int kChunkBytes = kBK * 128;          // one chunk of a block: 64 rows x 128 B
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kGatherWarps = 8;                 // warps 0-7
 constexpr int kMmaWarp = 8;
 constexpr int kEpiWarp0 = 12;                   // warps 12-15 = TMEM sub-partitions 0-3
@@ -50,9 +54,8 @@ constexpr uint32_t kColQ = 0;                   // Q: 288 columns (bf16 pairs)
 constexpr uint32_t kColS = 288;                 // S buffers: [288, 352), [352, 416)
 
 struct __align__(1024) Smem {
-  uint8_t kv[kStages][kChunks][kChunkBytes];    // 144 KB
+  uint8_t kv[kStages][kChunks][kChunkBytes];    // 216 KB
   int32_t rows[kMaxK];                          // KV row of every index entry (0 if invalid)
-  float p[kMaxK];                               // the target distribution, per entry
   float part[4][kBK];                           // per-warp head sums of one block
   uint32_t bmask[kMaxBlocks][2];                // valid entries of block b
   uint32_t mask[kMaxBlocks][2];                 // valid entries of the j-th non-empty block
@@ -66,6 +69,7 @@ struct __align__(1024) Smem {
   uint64_t mma_drain;
   uint32_t tmem_base;
 };
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory of one CTA on sm_100");
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -124,7 +128,6 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kl_kernel(const KlArgs a)
     fence_barrier_init();
     if (!q_ok) report(a.status, DSA_ERR_DEVICE_BOUNDS);
   }
-  for (int i = threadIdx.x; i < kMaxK; i += kThreads) S.p[i] = 0.f;
   if (warp == kMmaWarp) tmem_alloc(&S.tmem_base, kTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -289,6 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kl_kernel(const KlArgs a)
     }
     const float sl2 = a.scale_log2;
     const float l2 = a.lse[static_cast<int64_t>(qi) * kH + head] * 1.4426950408889634f;
+    float* const grow = a.grad + static_cast<int64_t>(qi) * a.ld_grad;
     bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
     // one block count for all four warps (read once, after the plan), so they
     // take the same named-barrier steps whatever their own waits did
@@ -327,8 +331,10 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kl_kernel(const KlArgs a)
       S.part[sub][2 * lane] = v[0];
       S.part[sub][2 * lane + 1] = v[1];
       named_bar_sync(2, 4 * 32);
+      // the target of the block's entries waits in the gradient row (global
+      // memory, L2-resident) until the final pass overwrites it with r - p
       if (et < kBK)
-        S.p[S.blk[j] * kBK + et] =
+        grow[S.blk[j] * kBK + et] =
             (S.part[0][et] + S.part[1][et] + S.part[2][et] + S.part[3][et]) * (1.f / kH);
       named_bar_sync(2, 4 * 32);
     }
@@ -360,12 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kl_kernel(const KlArgs a)
     z = (S.red[0][1] + S.red[1][1]) + (S.red[2][1] + S.red[3][1]);
     const float log_z = logf(z);
     float kl = 0.f;
-    float* grow = a.grad + static_cast<int64_t>(qi) * a.ld_grad;
+    __threadfence_block();   // every thread's targets in grow seen by the others
+    named_bar_sync(2, 4 * 32);
     for (int i = et; i < a.k; i += 128) {
       float g = 0.f;
       if (valid(i) && ok) {
         const float lr = (srow[i] - m) - log_z;     // log r_i
-        const float p = S.p[i];
+        const float p = grow[i];
         g = expf(lr) - p;
         if (p > 0.f) kl += p * (logf(p) - lr);
       }
