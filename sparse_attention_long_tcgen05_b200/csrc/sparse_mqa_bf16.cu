@@ -50,7 +50,8 @@
 // Roles per CTA (1024 threads, 8 warps per SM sub-partition):
 //   warps 0-15   plan (each scans two 64-entry blocks of the query's index row:
 //                physical rows, valid masks);
-//   warps 0-15, 17-19  copy the selected rows (all lanes, cp.async);
+//   warps 0-15, 17-18  copy the selected rows (all lanes, cp.async; three
+//                groups of six warps, each taking every third block);
 //   warp 16      owns TMEM and issues the MMAs;
 //   warps 20-23  softmax of the CTA's own heads (TMEM lanes 32s .. 32s+15);
 //   warps 24-27  send the peer's partial S (lanes 32s+16 .. 32s+31), as fp16;
@@ -78,11 +79,13 @@ constexpr int kChunkKV = kBK * 128;  // one 64-dim chunk of a key block: 64 rows
 constexpr int kMaxK = 2048;
 constexpr int kMaxBlocks = kMaxK / kBK;
 static_assert(kMaxBlocks <= 32, "one lane of a warp per key block in the plan's compaction");
-// Warp roles. 19 warps copy the selected rows (a block's 72 row-piece
-// instructions round-robin over them).
+// Warp roles. Three groups of six warps copy the selected rows (a block's 72
+// row-piece instructions round-robin over the warps of its group).
 constexpr int kPlanWarps = 16;       // warps 0-15 scan the index row (two blocks each)
 constexpr int kMmaWarp = 16;
-constexpr int kGatherIssuers = 19;   // warps 0-15 and 17-19 copy the selected rows
+constexpr int kGatherIssuers = 19;   // warps 0-15 and 17-19 (all meet on named barrier 2)
+constexpr int kGroups = 3;           // issuer groups, block j to group j % kGroups
+constexpr int kGroupWarps = 6;       // warps per group (issuer 18, warp 19, takes no block)
 constexpr int kSoftmaxWarp0 = 20;    // 20..23
 constexpr int kSendWarp0 = 24;       // 24..27
 constexpr int kRecvWarp0 = 28;       // 28..31
@@ -118,7 +121,7 @@ struct __align__(1024) Smem {
   float rx_l[64];                             // the peer's final row sums of its heads
   int32_t n_blocks;
   int32_t gather_n;                           // blocks the gather walks (issuer 0's view)
-  int32_t gather_go[2];                       // issuer 0: stage ready (1) or give up (0)
+  int32_t gather_go[kGroups][2];              // group leader: stage ready (1) or give up (0)
   uint64_t plan_full, q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t rope_full[kRopeStages], rope_empty[kRopeStages];
@@ -267,11 +270,11 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
     mbar_init(&S.plan_full, 1);
     mbar_init(&S.q_full, 12);          // softmax, send and receive warps (one arrival each)
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&S.kv_full[i], kGatherIssuers);   // one arrival per issuing warp
+      mbar_init(&S.kv_full[i], kGroupWarps);   // one arrival per warp of the block's group
       mbar_init(&S.kv_empty[i], 1);
     }
     for (int i = 0; i < kRopeStages; ++i) {
-      mbar_init(&S.rope_full[i], kGatherIssuers);
+      mbar_init(&S.rope_full[i], kGroupWarps);
       mbar_init(&S.rope_empty[i], 1);
     }
     mbar_init(&S.s_full, 1);
@@ -387,20 +390,23 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
       }
     }
     if (warp != kMmaWarp) {
-      // ---------------------------------------------------------- gather (19 issuing warps)
+      // ---------------------------------------------------------- gather (3 groups of 6 warps)
       // Block j's selected rows are copied with 16-byte cp.async straight into
       // the 128-byte-swizzled K-major tiles the MMAs read: the CTA's 256 value
       // columns of each of the 64 rows (one 512-byte row per warp instruction,
       // lane l copying 16 bytes of 64-dim chunk l / 8) and the 64 rope columns
       // of this CTA's 32 keys (four rows per instruction). The block's 72
-      // instructions go round-robin to the 19 issuing warps. A warp releases
-      // block j-1 to the MMA once its own copies of that block have landed (its
-      // cp.async groups), after a proxy fence that makes them visible to the
-      // tensor core; so each warp keeps two blocks of copies in flight.
-      // Only issuer 0 waits on the ring's barriers; the other 18 warps sleep on
-      // hardware named barrier 2 (taking no issue slots from the softmax warps)
-      // and learn from a shared flag whether to go on, so all 19 always take
-      // the same number of barrier steps.
+      // instructions go round-robin to the six warps of the block's group: 18
+      // of the 19 issuing warps form three groups, group g taking blocks
+      // j = g mod 3. A warp releases its block to the MMA as soon as its own
+      // copies of it have landed, after a proxy fence that makes them visible
+      // to the tensor core, so three blocks are in flight and no block waits
+      // for the next one to be issued (one group of 19 warps releasing block
+      // j-1 after issuing j: 134.8 ms at 128K; two groups 127.8; three 125.2).
+      // Only a group's first warp waits on the ring's barriers; the others
+      // sleep on the group's hardware named barrier (taking no issue slots from
+      // the softmax warps) and learn from a shared flag whether to go on, so
+      // all of a group's warps take the same number of barrier steps.
       const int issuer = warp < kMmaWarp ? warp : warp - 1;
       if (issuer == 0) {
         const bool ok = mbar_wait_warp(&S.plan_full, 0, a.status);
@@ -424,23 +430,25 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
           mbar_arrive(&S.rope_full[jj % kRopeStages]);
         }
       };
-      int issued = 0;
-      for (int j = 0; j < n; ++j) {
+      // Groups of issuing warps take every kGroups-th block; a group releases
+      // its block as soon as its own copies have landed, so no block waits for
+      // the issue of the next one.
+      const int grp = issuer / kGroupWarps;
+      const int li = issuer - grp * kGroupWarps;
+      for (int j = grp; j < n && grp < kGroups; j += kGroups) {
         const int st = j % kStages;
         const int rs = j % kRopeStages;
-        if (issuer == 0) {
+        const int use = (j / kGroups) & 1;
+        if (li == 0) {
           bool ok = mbar_wait_warp(&S.kv_empty[st], static_cast<uint32_t>((j / kStages) & 1) ^ 1u,
                                    a.status);
           if (ok)
             ok = mbar_wait_warp(&S.rope_empty[rs],
                                 static_cast<uint32_t>((j / kRopeStages) & 1) ^ 1u, a.status);
-          if (lane == 0) S.gather_go[j & 1] = ok ? 1 : 0;
+          if (lane == 0) S.gather_go[grp][use] = ok ? 1 : 0;
         }
-        named_bar_sync(2, kGatherIssuers * 32);
-        if (S.gather_go[j & 1] == 0) break;
-        // KV row of row r of block j: the planned row (sparse); dense, the
-        // key j*64 + r (clamped to the query's last key; masked past it) or
-        // slot r of the block's 64-token page
+        named_bar_sync(3 + grp, kGroupWarps * 32);
+        if (S.gather_go[grp][use] == 0) break;
         const int* rb = kDense ? nullptr : S.rows + S.blk[j] * kBK;
         int64_t dense_base = 0;
         if (kDense)
@@ -456,27 +464,22 @@ sparse_mqa_bf16_kernel(const __grid_constant__ AttnBf16Args a) {
         };
         const uint32_t kv_st = smem_u32(S.kv[st][c_l]);
         const uint32_t rope_st = smem_u32(S.rope[rs]);
-        for (int p = issuer; p < n_items; p += kGatherIssuers) {
+        for (int p = li; p < n_items; p += kGroupWarps) {
           if (p < kBK) {
-            const int r = p;                                   // row of the block
+            const int r = p;
             const char* src = kv_b + kv_row(r) * ld_b + val_off;
             cp_async16(kv_st + r * 128 + ((i_l ^ (r & 7)) << 4), src);
           } else {
-            const int rr = 4 * (p - kBK) + c_l;                // row of this CTA's 32 keys
+            const int rr = 4 * (p - kBK) + c_l;
             const char* src = kv_b + kv_row(32 * rank + rr) * ld_b + rope_off;
             cp_async16(rope_st + rr * 128 + ((i_l ^ (rr & 7)) << 4), src);
           }
         }
         cp_async_commit();
-        ++issued;
-        if (j > 0) {
-          cp_async_wait_group<1>();
-          release(j - 1);
-        }
+        cp_async_wait_group<0>();
+        release(j);
       }
-      // the last block, and a drain after a give-up: every copy lands first
       cp_async_wait_group<0>();
-      if (issued > 0) release(issued - 1);
     } else {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc_qk = make_idesc(kBK, 1, 1, 0, 0);   // bf16, A (TMEM) and B K-major
