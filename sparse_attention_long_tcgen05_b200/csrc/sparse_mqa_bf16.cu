@@ -86,6 +86,15 @@ constexpr int kMmaWarp = 16;
 constexpr int kGatherIssuers = 19;   // warps 0-15 and 17-19 (all meet on named barrier 2)
 constexpr int kGroups = 3;           // issuer groups, block j to group j % kGroups
 constexpr int kGroupWarps = 6;       // warps per group (issuer 18, warp 19, takes no block)
+// A group's leader starts block j once block j - kStages has left its ring
+// stage, waiting on the stage's barrier by phase parity. Its previous wait,
+// for block j - kGroups, ended after block j - kGroups - kStages had left, and
+// blocks leave in order, so block j - 2 kStages has left too when
+// kGroups <= kStages: the phase waited for is then the newest one with that
+// parity. With more groups than stages a wait could find an older completed
+// phase of the same parity and return before the stage is free.
+static_assert(kGroups <= kStages && kGroups <= kRopeStages,
+              "a copy group must not run two uses ahead on a ring stage");
 constexpr int kSoftmaxWarp0 = 20;    // 20..23
 constexpr int kSendWarp0 = 24;       // 24..27
 constexpr int kRecvWarp0 = 28;       // 28..31
