@@ -179,3 +179,34 @@ def test_bwd_full_size_sampled_rows(dsa, wl_index, n_rows):
     _close(dq_h, dq_ref, "dq")
     _check_dq_rows(dq_h, dq_ref, rows)
     _invariants(dkv, d_out, idx)
+
+
+def test_bwd_strided_index_and_dkv(dsa):
+    """An index row pitch larger than k and dkv rows wider than 576 floats: dq
+    equals the contiguous call's bit for bit, dkv (whose fp32 reductions land
+    in completion order) matches the oracle, and the padding of the wide dkv
+    rows is left untouched."""
+    L, k = 400, 192
+    wl = _wl(L, k)
+    inp = make_prefill(wl, device="cuda", seed=67)
+    idx = random_selection(L, L, k, device="cuda", seed=68)
+    d_out = make_grad_out(L, device="cuda", seed=69)
+    _, dq_ref_gpu, _, _ = _backward(dsa, inp.q, inp.kv, idx, k, d_out, wl.scale, L)
+    wide_idx = torch.full((L, k + 40), -7, dtype=torch.int32, device="cuda")
+    wide_idx[:, :k] = idx
+    att = dsa.attn_in(inp.q, inp.kv, wl.scale, 512)
+    out = torch.empty(L, 128, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(L, 128, device="cuda")
+    dsa.dsa_sparse_mqa_fwd(att, idx, k, out, lse)
+    dq = torch.empty(L, 128, 576, dtype=torch.bfloat16, device="cuda")
+    dkv_wide = torch.full((L, 640), 3.0, device="cuda")
+    dkv_wide[:, :576] = 0.0
+    delta = torch.empty(L, 128, 2, device="cuda")
+    dsa.dsa_sparse_mqa_bwd(att, wide_idx[:, :k], k, out, lse, d_out, dq, dkv_wide, delta)
+    assert dsa.dsa_check_status() == 0
+    assert torch.equal(dq, dq_ref_gpu)
+    assert torch.all(dkv_wide[:, 576:] == 3.0)
+    _, dkv_ref = O.sparse_mqa_backward(inp.q.double().cpu().numpy(), inp.kv.double().cpu().numpy(),
+                                       idx.cpu().numpy(), list(range(L)),
+                                       d_out.double().cpu().numpy(), wl.scale, 512)
+    _close(dkv_wide[:, :576].double().cpu().numpy(), dkv_ref, "dkv (wide rows)")
