@@ -333,7 +333,9 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kl_kernel(const KlArgs a)
       named_bar_sync(2, 4 * 32);
       // the target of the block's entries waits in the gradient row (global
       // memory, L2-resident) until the final pass overwrites it with r - p
-      if (et < kBK)
+      // (entries past k exist only in the last block's padding: nothing of
+      // them is stored, so a gradient row exactly k wide stays in bounds)
+      if (et < kBK && S.blk[j] * kBK + et < a.k)
         grow[S.blk[j] * kBK + et] =
             (S.part[0][et] + S.part[1][et] + S.part[2][et] + S.part[3][et]) * (1.f / kH);
       named_bar_sync(2, 4 * 32);

@@ -164,3 +164,28 @@ def test_kl_L32768_sampled_rows(libs):
     kv_sub, idx_local = T.gather_kv_rows(inp.kv, idx[r].cpu().numpy())
     _check(inp.q[r].double().cpu().numpy(), kv_sub, torch.from_numpy(idx_local).cuda(), sel[r],
            loss[r], grad[r], inp.wl.scale)
+
+
+def test_kl_ragged_k_tight_gradient_rows(libs):
+    """k = 100 (the last 64-key block holds 36 entries) with a gradient exactly
+    k wide: every row matches the oracle, and nothing is written past the last
+    row (a guard region after the buffer keeps its values)."""
+    dsa, T = libs
+    L, k = 300, 100
+    inp = make_prefill(_wl(L, k), device="cuda", seed=55)
+    ind, att = T.prefill_structs(inp)
+    ws = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_SELECT, ind, None, 0, 0, k))
+    idx = torch.empty(L, k, dtype=torch.int32, device="cuda")
+    sel = torch.empty(L, k, device="cuda")
+    dsa.dsa_select_scored(ind, k, idx, sel, ws)
+    out = torch.empty(L, 128, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(L, 128, device="cuda")
+    dsa.dsa_sparse_mqa_fwd(att, idx, k, out, lse)
+    loss = torch.empty(L, device="cuda")
+    buf = torch.full((L * k + 4096,), 7.0, device="cuda")
+    grad = buf[: L * k].view(L, k)
+    dsa.dsa_indexer_kl(att, idx, k, lse, sel, loss, grad)
+    assert dsa.dsa_check_status() == 0
+    assert torch.all(buf[L * k:] == 7.0)
+    _check(inp.q.double().cpu().numpy(), inp.kv.double().cpu().numpy(), idx, sel, loss, grad,
+           inp.wl.scale)
