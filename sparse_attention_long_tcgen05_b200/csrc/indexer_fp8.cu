@@ -32,7 +32,7 @@
 //             accumulator, and warps 2-5 reduce the first, warps 6-9 the
 //             second, so both halves of the epilogue work.
 //   warp 10   second paged producer (idle on contiguous keys)
-// A work unit is (group of G query rows, run of 16..32 key tiles of 128, 8..16
+// A work unit is (group of G query rows, run of 32..64 key tiles of 128, 8..16
 // with paged keys); the launcher picks the run length that spreads the units
 // most evenly over the CTAs. Launched after another kernel of the same selection, the kernel
 // starts at once and only the epilogue, which overwrites the score rows that
@@ -49,7 +49,7 @@ constexpr int kDim = 128;  // e4m3 bytes per head row / per key row
 constexpr int kKeyTile = 128;
 constexpr int kMaxG = 4;
 constexpr int kStages = 6;
-constexpr int kTilesPerUnit = 32;        // largest run of key tiles in a work unit
+constexpr int kTilesPerUnit = 64;        // largest run of key tiles in a work unit
 // Paged keys: the producer fetches a unit's page ids one per lane of a warp
 // (two 64-token pages per tile), so a paged unit spans at most 16 tiles.
 constexpr int kTilesPerUnitPaged = 16;
@@ -463,7 +463,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
 // whose units spread most evenly over the persistent CTAs, counting a unit's
 // set-up as half a tile. Longer runs cut the per-unit set-up (the query
 // group's load and the weights' staging): at 128K, runs of up to 32 tiles
-// instead of 16 took the indexer from 117.0 to 112.4 ms.
+// instead of 16 took the indexer from 117.0 to 112.5 ms, up to 64 to ~111.3.
 int balanced_tiles_per_unit(int n_groups, int n_tiles, int num_sms, int max_tpu) {
   int best = max_tpu;
   long long best_cost = -1;
