@@ -32,7 +32,7 @@
 //             accumulator, and warps 2-5 reduce the first, warps 6-9 the
 //             second, so both halves of the epilogue work.
 //   warp 10   second paged producer (idle on contiguous keys)
-// A work unit is (group of G query rows, run of 32..64 key tiles of 128, 8..16
+// A work unit is (group of G query rows, run of 8..64 key tiles of 128, 8..16
 // with paged keys); the launcher picks the run length that spreads the units
 // most evenly over the CTAs. Launched after another kernel of the same selection, the kernel
 // starts at once and only the epilogue, which overwrites the score rows that
@@ -50,10 +50,12 @@ constexpr int kKeyTile = 128;
 constexpr int kMaxG = 4;
 constexpr int kStages = 6;
 constexpr int kTilesPerUnit = 64;        // largest run of key tiles in a work unit
+constexpr int kMinTilesPerUnit = 8;      // shortest run the launcher considers
 // Paged keys: the producer fetches a unit's page ids one per lane of a warp
 // (two 64-token pages per tile), so a paged unit spans at most 16 tiles.
 constexpr int kTilesPerUnitPaged = 16;
 static_assert(2 * kTilesPerUnitPaged <= 32, "one lane of a warp per page id of a unit");
+static_assert(kMinTilesPerUnit <= kTilesPerUnitPaged, "a paged run can be the shortest");
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = 64 + kEpiThreads + 32;   // + warp 10, second paged producer
@@ -459,19 +461,22 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
 
 }  // namespace
 
-// Tiles per work unit: the run length (at most max_tpu, at least half of it)
-// whose units spread most evenly over the persistent CTAs, counting a unit's
-// set-up as half a tile. Longer runs cut the per-unit set-up (the query
-// group's load and the weights' staging): at 128K, runs of up to 32 tiles
-// instead of 16 took the indexer from 117.0 to 112.5 ms, up to 64 to ~111.3.
+// Tiles per work unit: the run length (kMinTilesPerUnit..max_tpu) whose units
+// spread most evenly over the persistent CTAs, counting a unit's set-up (the
+// query group's load and the weights' staging, during which the tensor pipe
+// waits) as one tile. Long runs pay the set-up less often: at 128K, runs of up
+// to 32 tiles instead of 16 took the indexer from 117.0 to 112.5 ms, up to 64
+// to 111.0. Short runs keep every SM busy when a block of rows has few key
+// tiles (148 rows near the start of a sequence form 37 groups: runs of 32
+// tiles there would leave three quarters of the SMs idle).
 int balanced_tiles_per_unit(int n_groups, int n_tiles, int num_sms, int max_tpu) {
   int best = max_tpu;
   long long best_cost = -1;
-  for (int tpu = max_tpu; tpu >= max_tpu / 2; --tpu) {
+  for (int tpu = max_tpu; tpu >= kMinTilesPerUnit; --tpu) {
     const long long units = static_cast<long long>(n_groups) * ((n_tiles + tpu - 1) / tpu);
     const long long grid = units < num_sms ? units : num_sms;
     const long long per_cta = (units + grid - 1) / grid;
-    const long long cost = per_cta * (2LL * (tpu < n_tiles ? tpu : n_tiles) + 1);
+    const long long cost = per_cta * ((tpu < n_tiles ? tpu : n_tiles) + 1);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = tpu;
