@@ -408,10 +408,7 @@ def run_ours(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3+bf16 (f32 accumulate)", "data": "synthetic",
-        "config": {"workload": wl.name, "L": L, "k": k, "H_I": wl.H_I, "d_I": wl.d_I,
-                   "H": wl.H, "d_qk": wl.D_K, "d_v": wl.D_V, "seed": "rank",
-                   "l2": "inputs larger than L2 (q alone 19.3 GB)",
-                   "parallelism": f"replicas x{world} (independent sequences)"},
+        "config": workload_config(wl, world),
         "roofline": roof, "rooflines": rooflines, "fp8_peak": fp8, "stages": stages,
         "cpu_baseline": cpu, "e2e": e2e, "cost_vs_position": curve, "indexer_kl": kl,
         "attention_backward": bwd,
@@ -605,6 +602,15 @@ def prefill_e2e(dsa, inp, ind, att, ws, idx, out, lse, k, args, world, n_chunks=
                    "calls, host<->device copies on two copy streams overlapping the kernels"}
 
 
+def workload_config(wl, world):
+    """The `config` object of a prefill line, shared by both arms."""
+    q_gb = wl.L * wl.H * wl.D_K * 2 / 1e9
+    return {"workload": wl.name, "L": wl.L, "k": wl.k, "H_I": wl.H_I, "d_I": wl.d_I,
+            "H": wl.H, "d_qk": wl.D_K, "d_v": wl.D_V, "seed": "rank",
+            "l2": f"inputs larger than L2 (q alone {q_gb:.1f} GB)",
+            "parallelism": f"replicas x{world} (independent sequences)"}
+
+
 def oracle_prefill_rate(inp, wl, budget_s=15.0, rows_cap=None):
     """The CPU oracle as it stands on a bounded sample of query rows of the same
     workload (uniform rows, so the mean prefix is ~L/2): tokens/s = rows/wall."""
@@ -733,26 +739,31 @@ def run_decode(args, world, rank, local, peaks, dsa, make_decode, wl):
 
 def run_reference(args, world, rank):
     """The oracle as it stands on the host cores: each step is a bounded sample
-    of query rows of the same workload; tokens/s = rows / wall time."""
+    of query rows of the same workload; tokens/s = rows / wall time, and
+    ms_per_step the mean wall time of a timed step (a sample, not the whole
+    workload)."""
     from sparse_attention_long_tcgen05_b200.inputs import WORKLOADS, make_prefill
     wl = next(w for w in WORKLOADS.values() if w.name == args.workload)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = make_prefill(wl, device=dev, seed=0)   # input generation only, untimed
-    rates = []
+    rates, walls = [], []
     for i in range(args.warmup + args.steps):
+        t0 = time.time()
         r = oracle_prefill_rate(inp, wl, budget_s=args.ref_step_s)
         if i >= args.warmup:
             rates.append(r)
+            walls.append(time.time() - t0)
     value = statistics.mean(r["value"] for r in rates)
     cpu = dict(rates[-1])
     cpu["value"] = value
     cpu["sample"] = (f"{args.steps} steps of ~{args.ref_step_s:.0f} s, each "
                      + rates[-1]["sample"])
     return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * statistics.mean(walls),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": wl.name, "L": wl.L, "k": wl.k},
+            "config": workload_config(wl, world),
             "cpu_baseline": cpu,
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
