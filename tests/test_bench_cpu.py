@@ -45,3 +45,31 @@ def test_workload_config_names_the_workload():
         assert c["parallelism"] == "replicas x2 (independent sequences)"
         q_gb = wl.L * 128 * 576 * 2 / 1e9
         assert f"{q_gb:.1f} GB" in c["l2"] and q_gb * 1e9 > 126e6   # q alone exceeds L2
+
+
+def _smi(sm, util, reasons=(), mx=1965, power=900):
+    """One nvidia-smi line of Clocks.FIELDS (csv, noheader, nounits)."""
+    act = ["Active" if n in reasons else "Not Active"
+           for n in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")]
+    return ", ".join(["0", str(sm), str(mx), str(power), str(util), "0x0"] + act) + "\n"
+
+
+def test_clock_summary_and_rejection():
+    idle = [_smi(345, 0, power=120)] * 3
+    # median SM clock under load; idle samples around the timed region ignored
+    c = bench.Clocks.parse(idle + [_smi(1965, 100), _smi(1950, 100), _smi(1965, 99)])
+    assert c["sm_mhz"] == 1965 and c["sm_max_mhz"] == 1965 and c["reasons"] == []
+    assert c["samples_under_load"] == 3 and c["power_w_max"] == 900
+    assert not bench.clock_rejected(c)
+    # the power cap is kept (and named); slowdowns reject the region
+    c = bench.Clocks.parse([_smi(1800, 100, ["sw_power_cap"])] * 4)
+    assert c["reasons"] == ["sw_power_cap"] and not bench.clock_rejected(c)
+    for why in bench.REJECTING_REASONS:
+        c = bench.Clocks.parse([_smi(1965, 100)] * 3 + [_smi(1200, 100, [why])])
+        assert why in c["reasons"] and bench.clock_rejected(c), why
+    # clocks held well below the maximum with no reason: a lock left behind
+    c = bench.Clocks.parse([_smi(1100, 100)] * 5)
+    assert c["reasons"] == [] and bench.clock_rejected(c)
+    # no samples (no nvidia-smi): nothing to reject
+    assert bench.Clocks.parse(["garbage\n"]) is None and not bench.clock_rejected(None)
+    assert bench.any_rank(True, 1) and not bench.any_rank(False, 1)

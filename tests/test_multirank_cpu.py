@@ -5,6 +5,8 @@ workload with no data exchange. Ranks meet only at barriers and at the
 max-over-ranks of the step time. These tests bring up two CPU ranks on
 127.0.0.1 and check the following:
 - every rank gets the slowest rank's time;
+- a clock rejection seen on one rank reaches every rank, so all time the step
+  again together;
 - the whole-job rate counts every rank's tokens;
 - the reference arm's other ranks exit at once, with no process group.
 """
@@ -35,7 +37,8 @@ def _rank_main(rank: int, world: int, port: int, q) -> None:
         backend = torch.distributed.get_backend()
         slow = bench.max_over_ranks(10.0 + 5.0 * rank, w)   # rank 1 is the slow one
         bench.barrier(w)
-        q.put((r, w, backend, slow, bench.job_rate(w, 131072, slow)))
+        again = (bench.any_rank(rank == 1, w), bench.any_rank(False, w))
+        q.put((r, w, backend, slow, bench.job_rate(w, 131072, slow), again))
     finally:
         torch.distributed.destroy_process_group()
 
@@ -57,10 +60,11 @@ def test_two_gloo_ranks_agree_on_the_slowest_time(monkeypatch):
             p.join()
     assert [p.exitcode for p in procs] == [0, 0]
     got = sorted(q.get(timeout=10) for _ in range(2))
-    for r, (rank, world, backend, slow, rate) in enumerate(got):
+    for r, (rank, world, backend, slow, rate, again) in enumerate(got):
         assert (rank, world, backend) == (r, 2, "gloo")
         assert slow == 15.0                          # max over ranks, on every rank
         assert rate == pytest.approx(2 * 131072 / 15e-3)
+        assert again == (True, False)                # rank 1's flag reaches rank 0
 
 
 def test_job_rate_is_whole_job_throughput():
