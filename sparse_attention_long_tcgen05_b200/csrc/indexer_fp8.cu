@@ -466,7 +466,7 @@ indexer_fp8_kernel(const __grid_constant__ IndexerFp8Args a, int G, int n_chunks
 // query group's load and the weights' staging, during which the tensor pipe
 // waits) as one tile. Long runs pay the set-up less often: at 128K, runs of up
 // to 32 tiles instead of 16 took the indexer from 117.0 to 112.5 ms, up to 64
-// to 111.0. Short runs keep every SM busy when a block of rows has few key
+// to 111.0 (up to 128 was slower again). Short runs keep every SM busy when a block of rows has few key
 // tiles (148 rows near the start of a sequence form 37 groups: runs of 32
 // tiles there would leave three quarters of the SMs idle).
 int balanced_tiles_per_unit(int n_groups, int n_tiles, int num_sms, int max_tpu) {
