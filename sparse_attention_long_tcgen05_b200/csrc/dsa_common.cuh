@@ -1,5 +1,5 @@
 // dsa_common.cuh -- sm_100a device primitives shared by the DSA kernels:
-// status reporting, bounded mbarrier waits, TMA tile/gather4 loads (never with
+// status reporting, bounded mbarrier waits, TMA tile loads (never with
 // cluster multicast), tcgen05 TMEM allocation / MMA / loads, UMMA shared-memory
 // and instruction descriptors, and cluster (DSMEM) helpers.
 #pragma once
@@ -254,19 +254,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
-// Four rows (y0..y3) of a 2-D tensor, x..x+box-1 columns each, into 4
-// consecutive box-sized rows of shared memory. The tensor map's box is one row.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int32_t x,
-                                            int32_t y0, int32_t y1, int32_t y2, int32_t y3,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
-      "r"(y2), "r"(y3)
       : "memory");
 }
 
